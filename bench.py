@@ -1,0 +1,564 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_2k|prefill_16k|decode_uniform|decode_shared_prefix]
+
+A step is one call of the entry point on one batch of the workload:
+  prefill_2k           attn_fwd, bf16 causal, B=4 H=16 N=2048 d=128   (default)
+  prefill_16k          attn_fwd, bf16 causal, B=1 H=32 N=16384 d=128 (x0.5)
+  decode_uniform       paged_attn_decode, 64 seqs, H=32, bs=16, L~U[128,4096]
+  decode_shared_prefix paged_attn_decode, 256 seqs, bs=32, 8-seq shared 512-token prefix
+The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
+decode_uniform, measured the same way in the same run, under "decode".
+
+Rates use algorithmic work: prefill FLOPs = 4 * B * H * d * (visible query-key
+pairs) (causal: N(N+1)/2 per head); decode bytes = K/V bytes the sequences
+attend over (sum_s L_s * 2 * H * d * 2; for the shared-prefix workload the
+unique physical bytes, logical bytes reported beside).
+
+Timing: W untimed warm-up steps, then K steps between barrier +
+cuda.synchronize, CUDA events on the launching stream around every launch;
+inputs rotate over copies whose total exceeds L2 (prefill) or exceed it alone
+(decode pools of GB).  Multi-GPU (torchrun): every rank runs its own replica
+(independent problems, weak scaling, no collective on the data path); the
+time is the max over ranks.  Only rank 0 prints the JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & paged-decode KV GB/s, as % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.25)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_sources_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "online_softmax_paged_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel sources are unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("sources") != kernel_sources_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- workloads
+
+class Prefill:
+    def __init__(self, cfg, name, device, seed=0):
+        self.name = name
+        self.cfg = cfg
+        self.B, self.H, self.N, self.d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+        self.causal = cfg["causal"]
+        one = 3 * self.B * self.H * self.N * self.d * 2
+        self.copies = max(1, math.ceil(3 * L2_BYTES / one))
+        self.sets = [W.dense_inputs(self.B, self.H, self.N, self.d, dtype=cfg["dtype"], mult=cfg["mult"],
+                                    seed=seed + i, device=device, causal=self.causal) for i in range(self.copies)]
+        self.O = torch.empty_like(self.sets[0]["Q"])
+        self.LSE = torch.empty((self.B, self.H, self.N), dtype=torch.float32, device=device)
+        pairs = self.N * (self.N + 1) // 2 if self.causal else self.N * self.N
+        self.work = 4.0 * self.B * self.H * self.d * pairs  # FLOP per step
+        self.unit, self.scale_unit = "TFLOP/s", 1e12
+        self.launches_per_step = 1
+        self.kernel = "prefill_bf16_kernel"
+
+    def step(self, i, osp):
+        s = self.sets[i % self.copies]
+        osp.attn_fwd(s["Q"], s["K"], s["V"], O=self.O, LSE=self.LSE, causal=self.causal, scale=s["scale"])
+
+    def config(self):
+        return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N, "d": self.d,
+                "causal": self.causal, "dtype": "bf16", "global_batch": self.B, "seq_len": self.N,
+                "l2": f"inputs rotate over {self.copies} copies ({self.copies * 3 * self.B * self.H * self.N * self.d * 2 / 2**20:.0f} MiB > L2)"}
+
+    def e2e(self, osp, steps, device):
+        s = self.sets[0]
+        hq, hk, hv = (s[k].cpu().pin_memory() for k in ("Q", "K", "V"))
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty(self.LSE.shape, dtype=torch.float32).pin_memory()
+        dq, dk, dv = torch.empty_like(s["Q"]), torch.empty_like(s["K"]), torch.empty_like(s["V"])
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            osp.attn_fwd(dq, dk, dv, O=self.O, LSE=self.LSE, causal=self.causal, scale=s["scale"])
+            ho.copy_(self.O, non_blocking=True)
+            hl.copy_(self.LSE, non_blocking=True)
+
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / steps
+        h2d = 3 * hq.numel() * hq.element_size()
+        d2h = ho.numel() * ho.element_size() + hl.numel() * 4
+        return ms, h2d, d2h
+
+    def cpu_sample(self, budget_s):
+        """The oracle on whole heads, one after another, until the budget."""
+        import numpy as np
+        import oracle
+        s = self.sets[0]
+        done, t0 = 0, time.perf_counter()
+        heads = [(b, h) for b in range(self.B) for h in range(self.H)]
+        for b, h in heads:
+            q, k, v = (s[x][b, h].float().cpu().numpy().astype(np.float64) for x in ("Q", "K", "V"))
+            oracle.attention_head(q, k, v, self.causal, s["scale"])
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return self.work * done / len(heads), dt, f"{done} of {len(heads)} (b, h) heads of {self.name}, full rows"
+
+
+class Decode:
+    def __init__(self, name, device, seed=0):
+        self.name = name
+        if name == "decode_uniform":
+            self.p = W.paged_uniform(device=device, seed=seed, **W.DECODE_UNIFORM)
+        else:
+            self.p = W.paged_shared_prefix(device=device, seed=seed, **W.DECODE_SHARED_PREFIX)
+        self.logical = W.logical_kv_bytes(self.p)
+        self.unique = W.unique_kv_bytes(self.p)
+        self.work = float(self.unique if name != "decode_uniform" else self.logical)  # bytes per step
+        self.O = torch.empty_like(self.p.q)
+        self.LSE = torch.empty(self.p.q.shape[:2], dtype=torch.float32, device=device)
+        import online_softmax_paged_b200 as osp
+        n = osp.paged_attn_decode_workspace_size(self.p.num_seqs, self.p.H, self.p.d, self.p.max_blocks_per_seq,
+                                                 self.p.block_size)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        self.ws_bytes = n
+        self.unit, self.scale_unit = "GB/s", 1e9
+        self.launches_per_step = 3
+        self.kernel = "decode_split_kernel"
+
+    def step(self, i, osp):
+        p = self.p
+        osp.paged_attn_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.block_size, O=self.O,
+                              LSE=self.LSE, scale=p.scale, workspace=self.ws)
+
+    def config(self):
+        p = self.p
+        c = {"workload": self.name, "num_seqs": p.num_seqs, "H": p.H, "d": p.d, "block_size": p.block_size,
+             "pool_blocks": p.num_blocks, "dtype": "bf16", "global_batch": p.num_seqs,
+             "seq_len": int(p.seq_lens.max().item()), "kv_bytes_logical": self.logical,
+             "kv_bytes_unique": self.unique,
+             "l2": f"KV pool {2 * p.k_cache.numel() * 2 / 2**30:.1f} GiB > L2"}
+        return c
+
+    def e2e(self, osp, steps, device):
+        p = self.p
+        hq = p.q.cpu().pin_memory()
+        ht = p.block_table.cpu().pin_memory()
+        hs = p.seq_lens.cpu().pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty(self.LSE.shape, dtype=torch.float32).pin_memory()
+        dq, dt, ds = torch.empty_like(p.q), torch.empty_like(p.block_table), torch.empty_like(p.seq_lens)
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            dq.copy_(hq, non_blocking=True)
+            dt.copy_(ht, non_blocking=True)
+            ds.copy_(hs, non_blocking=True)
+            osp.paged_attn_decode(dq, p.k_cache, p.v_cache, dt, ds, p.block_size, O=self.O, LSE=self.LSE,
+                                  scale=p.scale, workspace=self.ws)
+            ho.copy_(self.O, non_blocking=True)
+            hl.copy_(self.LSE, non_blocking=True)
+
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        h2d = hq.numel() * 2 + ht.numel() * 4 + hs.numel() * 4
+        d2h = ho.numel() * 2 + hl.numel() * 4
+        return e0.elapsed_time(e1) / steps, h2d, d2h
+
+    def cpu_sample(self, budget_s):
+        import numpy as np
+        import oracle
+        p = self.p
+        sl = p.seq_lens.cpu().numpy()
+        bt = p.block_table.cpu().numpy()
+        q = p.q.float().cpu().numpy().astype(np.float64)
+
+        class Lazy:
+            def __init__(self, t):
+                self.t, self.shape = t, tuple(t.shape)
+
+            def __getitem__(self, i):
+                return self.t[int(i)].float().cpu().numpy()
+
+        kc, vc = Lazy(p.k_cache), Lazy(p.v_cache)
+        done_bytes, n, t0 = 0, 0, time.perf_counter()
+        for s in range(p.num_seqs):
+            oracle.paged_decode(q, kc, vc, bt, sl, p.block_size, p.scale, seqs=[s])
+            done_bytes += int(sl[s]) * 2 * p.H * p.d * 2
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return float(done_bytes), dt, f"{n} of {p.num_seqs} sequences of {self.name} (all heads)"
+
+
+def make_workload(name, device, seed=0):
+    if name == "prefill_2k":
+        return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
+    if name == "prefill_16k":
+        return Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
+    if name in ("decode_uniform", "decode_shared_prefix"):
+        return Decode(name, device, seed)
+    raise SystemExit(f"unknown workload {name}")
+
+
+# ---------------------------------------------------------------- timing
+
+def time_steps(wl, osp, steps, warmup, device, ws):
+    st = torch.cuda.current_stream(device)
+    for i in range(warmup):
+        wl.step(i, osp)
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize(device)
+    t_region0 = time.perf_counter()
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(st)
+    for i in range(steps):
+        evs[i][0].record(st)
+        wl.step(warmup + i, osp)
+        evs[i][1].record(st)
+    g1.record(st)
+    torch.cuda.synchronize(device)
+    barrier(ws)
+    wall = time.perf_counter() - t_region0
+    per = [a.elapsed_time(b) for a, b in evs]
+    total_ms = g0.elapsed_time(g1)
+    return per, total_ms, wall
+
+
+def roofline(wl, per_ms, pk, pk_src, bound):
+    launch_ms = statistics.mean(per_ms)
+    achieved = wl.work / (launch_ms * 1e-3) / wl.scale_unit
+    if bound == "tensor":
+        peak = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        unit = "TFLOP/s"
+    else:
+        peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        unit = "GB/s"
+    tr = recorded_traffic(wl.kernel, wl.name)
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": tr, "peak_source": pk_src,
+            "kernel": wl.kernel, "launch_ms": round(launch_ms, 5)}
+
+
+def run_ours(args):
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import online_softmax_paged_b200 as osp
+    osp.load()
+    pk, pk_src = peaks()
+
+    wl = make_workload(args.workload, device, seed=args.seed + rank)
+    bound = "tensor" if isinstance(wl, Prefill) else "hbm"
+    with ClockSampler(local) as clocks:
+        per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws)
+    t_max = max_over_ranks(total_ms, ws)
+    work_all = sum_over_ranks(wl.work * args.steps, ws)
+    value = work_all / (t_max * 1e-3) / wl.scale_unit
+    rl = roofline(wl, per, pk, pk_src, bound)
+
+    e2e_ms, h2d, d2h = wl.e2e(osp, max(3, min(args.steps, 20)), device)
+    e2e_ms = max_over_ranks(e2e_ms, ws)
+    e2e_val = sum_over_ranks(wl.work, ws) / (e2e_ms * 1e-3) / wl.scale_unit
+
+    extra = {}
+    if args.workload == "prefill_2k" and not args.no_decode:
+        dec = make_workload("decode_uniform", device, seed=args.seed + rank)
+        per_d, total_d, _ = time_steps(dec, osp, args.steps, args.warmup, device, ws)
+        td = max_over_ranks(total_d, ws)
+        extra["decode"] = {"workload": "decode_uniform", "value": round(sum_over_ranks(dec.work * args.steps, ws)
+                                                                        / (td * 1e-3) / 1e9, 2),
+                           "unit": "GB/s", "ms_per_step": round(td / args.steps, 5),
+                           "roofline": roofline(dec, per_d, pk, pk_src, "hbm"), "config": dec.config(),
+                           "gpu_launches": dec.launches_per_step * args.steps}
+        del dec
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        work, dt, sample = wl.cpu_sample(args.cpu_budget)
+        cpu = {"value": round(work / dt / wl.scale_unit, 6), "unit": wl.unit, "cores": _cpu_threads(),
+               "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16)",
+                "config": {**wl.config(), "parallelism": f"replicas{ws}" if ws > 1 else "single"},
+                "roofline": rl, "cpu_baseline": cpu,
+                "e2e": {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+                "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks.summary(),
+                "timed_wall_s": round(wall, 3), **extra}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    """The oracle (plain fp64 CPU code, as it stands) on the same workload,
+    one bounded sample per step; rank 0 only."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    name = args.workload
+    if name.startswith("prefill"):
+        cfg = W.PREFILL_CAUSAL_2K if name == "prefill_2k" else W.PREFILL_CAUSAL_16K
+        B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+        pairs = N * (N + 1) // 2
+        per_head = 4.0 * d * pairs
+        unit, su = "TFLOP/s", 1e12
+        inp = W.dense_inputs(B, H, N, d, dtype=cfg["dtype"], mult=cfg["mult"], seed=args.seed, device=dev,
+                             causal=True)
+        heads = [(b, h) for b in range(B) for h in range(H)]
+
+        def one(i):
+            b, h = heads[i % len(heads)]
+            q, k, v = (inp[x][b, h].float().cpu().numpy().astype(np.float64) for x in ("Q", "K", "V"))
+            oracle.attention_head(q, k, v, True, inp["scale"])
+            return per_head
+
+        sample = f"one (b, h) head of {name} per step"
+        config = {"workload": name, "B": B, "H": H, "N": N, "d": d, "causal": True, "dtype": "bf16",
+                  "global_batch": B, "seq_len": N}
+    else:
+        wl = Decode(name, dev, args.seed)
+        p = wl.p
+        sl = p.seq_lens.cpu().numpy()
+        bt = p.block_table.cpu().numpy()
+        q = p.q.float().cpu().numpy().astype(np.float64)
+        unit, su = "GB/s", 1e9
+        kc_t, vc_t = p.k_cache, p.v_cache
+
+        class Lazy:
+            def __init__(self, t):
+                self.t, self.shape = t, tuple(t.shape)
+
+            def __getitem__(self, i):
+                return self.t[int(i)].float().cpu().numpy()
+
+        def one(i):
+            s = i % p.num_seqs
+            oracle.paged_decode(q, Lazy(kc_t), Lazy(vc_t), bt, sl, p.block_size, p.scale, seqs=[s])
+            return float(int(sl[s]) * 2 * p.H * p.d * 2)
+
+        sample = f"one sequence of {name} per step (all heads)"
+        config = wl.config()
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    work = 0.0
+    for i in range(args.steps):
+        work += one(args.warmup + i)
+    dt = time.perf_counter() - t0
+    val = work / dt / su
+    line = {"metric": METRIC, "value": round(val, 6), "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16)",
+            "impl": "reference", "config": config,
+            "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_2k",
+                    choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode leg of the default line")
+    args = ap.parse_args(argv)
+    if args.impl == "ours":
+        args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention forward library.
+ *
+ * Two entry points compute O = softmax(scale * Q K^T) V with online softmax
+ * (a running max m and sum l per query row, the O accumulator rescaled as new
+ * key tiles arrive) and emit the per-row logsumexp:
+ *
+ *   attn_fwd           dense prefill, causal or not, [B, H, N, d] tensors.
+ *   paged_attn_decode  one query token per sequence; keys and values are read
+ *                      from a paged KV cache through a per-sequence block
+ *                      table of fixed-size blocks.
+ *
+ * Sources:
+ *   "一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解",
+ *     section 一 (standard self-attention; formula image lost, read as
+ *     softmax(Q K^T / sqrt(d)) V), section 二 核心原理 (tiling, safe softmax,
+ *     stored statistics), section 二 FlashAttention-2 改进 (keep only the
+ *     logsumexp), section 三 核心原理 (blocks of 16 or 32 tokens, block table
+ *     from contiguous logical to non-contiguous physical blocks).
+ *   "第 2 章核心模块：FlashAttention-2 与 PagedAttention 实现解析",
+ *     section 2.1 (incremental normalisation), section 2.2 (paged loop).
+ *   "Transformer内存优化：从Flash Attention到Page Attention", section 1.1
+ *     (layout [batch, heads, seq_len, dim]).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory and keeps no pointer after return.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream); nothing
+ *     synchronises the host.  Outputs are valid once the stream reaches the
+ *     launch.
+ *   - Tensors are contiguous, row-major, in the shapes stated, and 16-byte
+ *     aligned.  Inputs are read-only; outputs are written completely.
+ *   - Host-side argument checks run before any launch and return
+ *     ATTN_EINVAL or ATTN_EUNSUPPORTED with nothing launched.  A failed launch
+ *     returns ATTN_ECUDA.  Problems only the device can see (a block-table
+ *     entry out of range, a sequence length out of range, a pipeline wait
+ *     that exceeded its iteration limit) are OR-ed into `*err_flag` (a
+ *     caller-zeroed device int32, may be NULL) as ATTN_DEVERR_* bits; the
+ *     kernels never trap.  attn_read_error() turns the flag into a status.
+ *   - LSE is the natural logarithm of sum_j exp(scale * q . k_j), fp32.
+ */
+#ifndef ONLINE_SOFTMAX_PAGED_ATTN_H
+#define ONLINE_SOFTMAX_PAGED_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *attn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_EINVAL = 1,       /* bad pointer, size, alignment or shape */
+    ATTN_EUNSUPPORTED = 2, /* valid but not implemented (head dim, dtype) */
+    ATTN_ECUDA = 3,        /* a CUDA runtime / driver call failed */
+    ATTN_EDEVICE = 4       /* the device reported a problem via err_flag */
+} attn_status;
+
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/* Bits the kernels OR into *err_flag. */
+#define ATTN_DEVERR_BLOCK_TABLE 1 /* block_table entry outside [0, num_blocks) */
+#define ATTN_DEVERR_SEQ_LEN 2     /* seq_len < 0 or > max_blocks_per_seq * block_size */
+#define ATTN_DEVERR_TIMEOUT 4     /* a pipeline wait exceeded its iteration limit */
+
+/*
+ * Dense attention forward (prefill).
+ *
+ * Q, K, V, O : [B, H, N, d] of `dt` (ATTN_BF16 or ATTN_F32).
+ * LSE        : [B, H, N] fp32.
+ * causal     : nonzero -> query row i sees keys 0..i (square, Nq = Nk = N).
+ * scale      : multiplies q . k (normally 1/sqrt(d)); must be finite and > 0.
+ * Supported  : d in {64, 128}; N >= 1; B * H >= 1.  bf16 runs on the
+ *              tcgen05 tensor cores with fp32 accumulation (P is rounded to
+ *              bf16 before the P V product); fp32 runs on CUDA cores in fp32.
+ * err_flag   : optional device int32, see the conventions above.
+ * Result     : O_i = sum_j softmax_j(scale q_i . k_j) v_j in `dt`,
+ *              LSE_i = ln sum_j exp(scale q_i . k_j).
+ */
+ATTN_API attn_status attn_fwd(const void *Q, const void *K, const void *V, void *O, float *LSE,
+                     int B, int H, int N, int d, int causal, float scale,
+                     attn_dtype dt, int32_t *err_flag, attn_stream_t stream);
+
+/*
+ * Bytes of device workspace paged_attn_decode needs for these sizes (split-KV
+ * partial outputs and their logsumexps).  Returns 0 for invalid sizes.
+ */
+ATTN_API size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq,
+                                        int block_size);
+
+/*
+ * Tokens per split-KV chunk the decode uses for these sizes (a function of
+ * the sizes only, never of the data; exposed for tests and tooling).
+ */
+ATTN_API int paged_attn_decode_split_tokens(int num_seqs, int H, int d, int max_blocks_per_seq,
+                                   int block_size);
+
+/*
+ * Paged decode: one query token per sequence against its cached keys/values.
+ *
+ * q            : [num_seqs, H, d] bf16.
+ * k_cache,
+ * v_cache      : [num_blocks, H, block_size, d] bf16 (a block holds
+ *                block_size consecutive tokens of one sequence, all heads).
+ * block_table  : int32 [num_seqs, max_blocks_per_seq]; entry [s][lb] is the
+ *                physical block holding logical block lb (tokens
+ *                lb*block_size ..) of sequence s.  Entries past a sequence's
+ *                last block are never read.  Several sequences may name the
+ *                same physical block (shared prefix, read-only).
+ * seq_lens     : int32 [num_seqs]; the number of cached tokens the query
+ *                attends to (its own token included if it was written).
+ * O            : [num_seqs, H, d] bf16.   LSE : [num_seqs, H] fp32.
+ * workspace    : device buffer of at least
+ *                paged_attn_decode_workspace_size(...) bytes, 16-byte
+ *                aligned, contents ignored on entry and clobbered.
+ * Supported    : bf16; d = 128; block_size in {16, 32}.
+ * Device checks: a block-table entry outside [0, num_blocks) or a seq_len
+ *                outside [0, max_blocks_per_seq * block_size] sets the
+ *                matching ATTN_DEVERR_* bit; that sequence's O is written as
+ *                0 and its LSE as -inf, and no out-of-range address is read.
+ * seq_len == 0 : O = 0, LSE = -inf (no error).
+ * Determinism  : the split plan and every reduction order depend only on the
+ *                logical token positions, so moving blocks to other physical
+ *                ids (with a matching table) gives bit-identical results.
+ */
+ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_table, const int32_t *seq_lens, int block_size,
+                              void *O, float *LSE,
+                              int num_seqs, int H, int d, int num_blocks, int max_blocks_per_seq,
+                              float scale, attn_dtype dt, void *workspace, size_t workspace_bytes,
+                              int32_t *err_flag, attn_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the device int32 at err_flag and return
+ * ATTN_OK if it is 0, ATTN_EDEVICE otherwise (the bits are written to
+ * *bits_out when it is not NULL).  The flag is not reset.
+ */
+ATTN_API attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+ATTN_API const char *attn_status_str(attn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ONLINE_SOFTMAX_PAGED_ATTN_H */

@@ -1,0 +1,174 @@
+"""Python binding of the sm_100a exact-attention library (``include/attn.h``).
+
+Argument marshalling only: every step of attention runs in the CUDA kernels
+of ``libattn_sm100.so``.  PyTorch supplies device memory and the stream.
+There is no fallback: if the library is missing or a tensor is not on a CUDA
+device the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "AttnError", "attn_fwd", "paged_attn_decode", "paged_attn_decode_workspace_size",
+    "paged_attn_decode_split_tokens", "attn_read_error", "attn_status_str", "lib_path", "load",
+    "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libattn_sm100.so")
+
+ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_ECUDA, ATTN_EDEVICE = range(5)
+ATTN_F32, ATTN_BF16 = 0, 1
+ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT = 1, 2, 4
+
+# every function include/attn.h declares
+EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
+                    "paged_attn_decode", "attn_read_error", "attn_status_str")
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {attn_status_str(status)} (status {status})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m online_softmax_paged_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32p, fp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p
+    c_int, c_float, c_size = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, fp, c_int, c_int, c_int, c_int, c_int, c_float, c_int, vp, vp]
+    lib.attn_fwd.restype = c_int
+    lib.paged_attn_decode_workspace_size.argtypes = [c_int] * 5
+    lib.paged_attn_decode_workspace_size.restype = c_size
+    lib.paged_attn_decode_split_tokens.argtypes = [c_int] * 5
+    lib.paged_attn_decode_split_tokens.restype = c_int
+    lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
+                                      c_float, c_int, vp, c_size, vp, vp]
+    lib.paged_attn_decode.restype = c_int
+    lib.attn_read_error.argtypes = [vp, i32p, vp]
+    lib.attn_read_error.restype = c_int
+    lib.attn_status_str.argtypes = [c_int]
+    lib.attn_status_str.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def attn_status_str(status: int) -> str:
+    return load().attn_status_str(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be on a CUDA device (the library has no CPU path)")
+
+
+def _dtype_code(dt):
+    if dt == torch.bfloat16:
+        return ATTN_BF16
+    if dt == torch.float32:
+        return ATTN_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def attn_fwd(Q, K, V, O=None, LSE=None, causal=False, scale=None, err_flag=None, stream=None):
+    """Dense attention forward.  Q, K, V: [B, H, N, d] contiguous CUDA tensors of
+    one dtype (bf16 or fp32).  Returns (O, LSE); O and LSE are allocated when
+    not given.  See ``attn_fwd`` in include/attn.h for the contract."""
+    _check_cuda(Q, K, V, O, LSE, err_flag)
+    B, H, N, d = Q.shape
+    if K.shape != Q.shape or V.shape != Q.shape or K.dtype != Q.dtype or V.dtype != Q.dtype:
+        raise ValueError("Q, K, V must share shape and dtype")
+    if not (Q.is_contiguous() and K.is_contiguous() and V.is_contiguous()):
+        raise ValueError("Q, K, V must be contiguous")
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = load().attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, int(bool(causal)),
+                         float(scale), _dtype_code(Q.dtype), _ptr(err_flag), _stream(stream, Q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return O, LSE
+
+
+def paged_attn_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq, block_size) -> int:
+    return int(load().paged_attn_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq, block_size))
+
+
+def paged_attn_decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size) -> int:
+    return int(load().paged_attn_decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size))
+
+
+def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=None, LSE=None, scale=None,
+                      workspace=None, err_flag=None, stream=None):
+    """Paged decode.  q [S, H, d] bf16; caches [num_blocks, H, block_size, d]
+    bf16; block_table int32 [S, max_blocks_per_seq]; seq_lens int32 [S].
+    Returns (O, LSE).  ``workspace`` (uint8 CUDA tensor) is allocated when
+    not given.  See ``paged_attn_decode`` in include/attn.h."""
+    _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, workspace, err_flag)
+    S, H, d = q.shape
+    num_blocks = k_cache.shape[0]
+    mb = block_table.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if k_cache.shape != v_cache.shape or k_cache.shape[1] != H or k_cache.shape[2] != block_size or \
+            k_cache.shape[3] != d:
+        raise ValueError("caches must be [num_blocks, H, block_size, d]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((S, H), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = paged_attn_decode_workspace_size(S, H, d, mb, block_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load().paged_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                  int(block_size), _ptr(O), _ptr(LSE), S, H, d, num_blocks, mb, float(scale),
+                                  _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _ptr(err_flag), _stream(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_attn_decode")
+    return O, LSE
+
+
+def attn_read_error(err_flag, stream=None) -> int:
+    """Synchronise the stream and return the device error bits (0 = none)."""
+    bits = ctypes.c_int32(0)
+    st = load().attn_read_error(_ptr(err_flag), ctypes.byref(bits), _stream(stream, err_flag.device))
+    if st not in (ATTN_OK, ATTN_EDEVICE):
+        raise AttnError(st, "attn_read_error")
+    return int(bits.value)

@@ -1,0 +1,94 @@
+// api.cu -- the extern "C" boundary declared in include/attn.h: argument
+// checks, dispatch to the sm_100a kernels, status codes.  No allocation, no
+// host synchronisation (except attn_read_error, which exists to sync).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/attn.h"
+#include "launch.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void *Q, const void *K, const void *V, void *O, float *LSE, int B, int H, int N, int d,
+                     int causal, float scale, attn_dtype dt, int32_t *err_flag, attn_stream_t stream) {
+    if (!Q || !K || !V || !O || !LSE) return ATTN_EINVAL;
+    if (B < 1 || H < 1 || N < 1) return ATTN_EINVAL;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
+    if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
+    if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return ATTN_EINVAL;
+    if ((long long)B * H > 0x7fffffffLL / 2) return ATTN_EINVAL;
+    if (dt == ATTN_F32 && (H > 65535 || B > 65535)) return ATTN_EINVAL;
+    osp::DenseLaunch p{Q, K, V, O, LSE, B, H, N, d, causal ? 1 : 0, scale, err_flag};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dt == ATTN_BF16 ? osp::launch_prefill_bf16(p, s) : osp::launch_dense_f32(p, s);
+}
+
+size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq, int block_size) {
+    if (num_seqs < 0 || H < 1 || d != 128 || max_blocks_per_seq < 1 || block_size < 16 || block_size % 16)
+        return 0;
+    return osp::decode_workspace_bytes(num_seqs, H, d, max_blocks_per_seq, block_size);
+}
+
+int paged_attn_decode_split_tokens(int num_seqs, int H, int d, int max_blocks_per_seq, int block_size) {
+    if (num_seqs < 0 || H < 1 || d != 128 || max_blocks_per_seq < 1 || block_size < 16 || block_size % 16)
+        return 0;
+    return osp::decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size);
+}
+
+attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                              const int32_t *seq_lens, int block_size, void *O, float *LSE, int num_seqs, int H,
+                              int d, int num_blocks, int max_blocks_per_seq, float scale, attn_dtype dt,
+                              void *workspace, size_t workspace_bytes, int32_t *err_flag, attn_stream_t stream) {
+    if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
+    if (num_seqs < 0 || H < 1 || num_blocks < 1 || max_blocks_per_seq < 1) return ATTN_EINVAL;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
+    if (dt != ATTN_BF16) return ATTN_EUNSUPPORTED;
+    if (d != 128) return ATTN_EUNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return ATTN_EUNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return ATTN_EINVAL;
+    if ((long long)num_blocks * H * block_size * d > (1LL << 46)) return ATTN_EINVAL;
+    if (num_seqs == 0) return ATTN_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !O || !LSE || !workspace) return ATTN_EINVAL;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(O) || !aligned16(workspace))
+        return ATTN_EINVAL;
+    if (((uintptr_t)block_table & 3u) || ((uintptr_t)seq_lens & 3u) || ((uintptr_t)LSE & 3u)) return ATTN_EINVAL;
+    if ((long long)num_seqs * H > 0x7fffffffLL / 4) return ATTN_EINVAL;
+    if (workspace_bytes < osp::decode_workspace_bytes(num_seqs, H, d, max_blocks_per_seq, block_size))
+        return ATTN_EINVAL;
+    osp::DecodeLaunch p{q,        k_cache,  v_cache, block_table, seq_lens,         O,          LSE,
+                        num_seqs, H,        d,       num_blocks,  max_blocks_per_seq, block_size, scale,
+                        workspace, err_flag};
+    return osp::launch_paged_decode(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream) {
+    if (!err_flag) return ATTN_EINVAL;
+    int32_t v = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, err_flag, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ATTN_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ECUDA;
+    if (bits_out) *bits_out = v;
+    return v ? ATTN_EDEVICE : ATTN_OK;
+}
+
+const char *attn_status_str(attn_status s) {
+    switch (s) {
+        case ATTN_OK: return "ok";
+        case ATTN_EINVAL: return "invalid argument";
+        case ATTN_EUNSUPPORTED: return "unsupported configuration";
+        case ATTN_ECUDA: return "CUDA error";
+        case ATTN_EDEVICE: return "device-side error reported in err_flag";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,451 @@
+// decode_paged.cu -- paged-KV decode for sm_100a: one query token per
+// sequence, keys/values gathered through a per-sequence block table.
+//
+// Method (pages): "第 2 章核心模块：FlashAttention-2 与 PagedAttention 实现解析"
+// section 2.2 -- for each logical block look up the physical block, fetch
+// only that block's K/V, score it and merge into the running max/sum;
+// section 2.1 -- the incremental normalisation (running max m, running sum l,
+// correct the accumulated O).  "一文掌握大模型推理加速：FlashAttention与
+// PagedAttention技术详解" section 三 核心原理 -- fixed blocks of 16 or 32
+// tokens, contiguous logical / non-contiguous physical blocks.
+//
+// B200 design (HBM-bound: ~1 flop per byte):
+//   1. plan kernel      -- one CTA scans seq_lens into per-sequence split
+//                          offsets (split size fixed by the host from the
+//                          sizes only) and zeroes the work counter.
+//   2. split kernel     -- persistent, one CTA per SM, every warp an
+//                          independent worker.  A warp takes (sequence, split,
+//                          head) items from an atomic counter and streams the
+//                          split's 16-token K and V tiles (4 KiB each,
+//                          contiguous inside a block) into its own ring of
+//                          shared-memory slots with 1-D bulk async copies
+//                          completing on per-slot mbarriers.  Math reads the
+//                          slots with 16-byte vector loads: a half-warp holds
+//                          one 128-wide row (8 dims per lane), q.k is reduced
+//                          with warp shuffles, and the online-softmax update is
+//                          applied once per tile.  Each item writes a
+//                          normalised partial O and its log2-sum-exp.
+//   3. merge kernel     -- per sequence: validate the table, then
+//                          LSE = log sum_p exp(LSE_p), O = sum_p e^{LSE_p-LSE} O_p.
+// Every arithmetic order depends only on logical token positions, so moving
+// blocks to other physical ids gives bit-identical results.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace osp {
+namespace {
+
+constexpr int kD = 128;                         // head dim supported here
+constexpr int kTileTok = 16;                    // tokens per pipeline tile
+constexpr int kTileBytes = kTileTok * kD * 2;   // 4 KiB of K (or of V)
+constexpr int kWarps = 8;                       // workers per CTA
+constexpr int kStages = 3;                      // ring slots per worker
+constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
+constexpr int kSmemBytes = kWarps * kStages * kSlotBytes + kWarps * kStages * 8 + 64;
+
+struct DecodeArgs {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_cache;
+    const __nv_bfloat16 *v_cache;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    __nv_bfloat16 *O;
+    float *LSE;
+    int32_t *err;
+    // workspace views
+    int32_t *counter;     // [1]
+    int32_t *item_start;  // [num_seqs + 1] prefix sum of splits per sequence
+    float *part_lse;      // [num_seqs, H, max_splits] log2 units
+    float *part_o;        // [num_seqs, H, max_splits, d] normalised
+    int num_seqs, H, num_blocks, max_blocks, block_size, split_tokens, max_splits;
+    float scale_log2;     // scale * log2(e)
+};
+
+__device__ __forceinline__ bool seq_len_ok(int L, const DecodeArgs &a) {
+    return L >= 0 && (long long)L <= (long long)a.max_blocks * a.block_size;
+}
+
+// ------------------------------------------------------------------ plan
+
+__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) {
+        carry = 0;
+        *a.counter = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < a.num_seqs; base += 1024) {
+        const int s = base + tid;
+        int n = 0;
+        if (s < a.num_seqs) {
+            const int L = a.seq_lens[s];
+            if (seq_len_ok(L, a)) n = (L + a.split_tokens - 1) / a.split_tokens;
+        }
+        int x = n;  // inclusive warp scan
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int w = warp_tot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_tot[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const int excl = carry + (wid ? warp_tot[wid - 1] : 0) + x - n;
+        if (s < a.num_seqs) a.item_start[s] = excl;
+        __syncthreads();
+        if (tid == 1023) carry = excl + n;
+        __syncthreads();
+    }
+    if (tid == 0) a.item_start[a.num_seqs] = carry;
+}
+
+// ------------------------------------------------------------------ split
+
+struct WarpRing {
+    uint8_t *slots;   // kStages * kSlotBytes
+    uint64_t *full;   // kStages barriers
+};
+
+// Physical id of the block holding logical token `tok` of sequence s, or -1
+// (with the error bit set) when the table entry is out of range.
+__device__ __forceinline__ int resolve_block(const DecodeArgs &a, int s, int tok) {
+    const int lb = tok / a.block_size;
+    const int phys = __ldg(a.block_table + (size_t)s * a.max_blocks + lb);
+    return (phys >= 0 && phys < a.num_blocks) ? phys : -1;
+}
+
+__device__ __forceinline__ size_t tile_offset(const DecodeArgs &a, int phys, int h, int tok) {
+    // element offset of token `tok` of head h inside physical block phys
+    return (((size_t)phys * a.H + h) * a.block_size + (tok % a.block_size)) * kD;
+}
+
+// Lane 0: start the copy of tile `t` (tokens tok0 + 16 t ..) into slot.
+__device__ __forceinline__ void issue_tile(const DecodeArgs &a, const WarpRing &r, int slot, int s, int h,
+                                           int tok) {
+    const int phys = resolve_block(a, s, tok);
+    uint64_t *bar = r.full + slot;
+    if (phys < 0) {
+        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+        mbar_arrive(bar);  // complete the phase without touching memory
+        return;
+    }
+    const size_t off = tile_offset(a, phys, h, tok);
+    uint8_t *dst = r.slots + slot * kSlotBytes;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, kSlotBytes);
+    bulk_g2s(dst, a.k_cache + off, kTileBytes, bar);
+    bulk_g2s(dst + kTileBytes, a.v_cache + off, kTileBytes, bar);
+}
+
+__global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    WarpRing ring;
+    ring.slots = smem + (size_t)wid * kStages * kSlotBytes;
+    ring.full = reinterpret_cast<uint64_t *>(smem + kWarps * kStages * kSlotBytes) + wid * kStages;
+    if (lane == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(ring.full + i, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    const int half = lane >> 4, li = lane & 15;
+    const int total = a.item_start[a.num_seqs] * a.H;
+    uint32_t gtile = 0;  // tiles consumed by this warp so far (ring phase)
+    uint32_t pending = 0;  // lane 0: slots with a copy in flight
+    bool dead = false;
+    int s_hint = 0;
+
+    while (!dead) {
+        int item = 0;
+        if (lane == 0) item = atomicAdd(a.counter, 1);
+        item = __shfl_sync(0xffffffffu, item, 0);
+        if (item >= total) break;
+        const int k = item / a.H, h = item - k * a.H;
+        // sequence holding split k: item_start[s] <= k < item_start[s + 1]
+        int lo = 0, hi = a.num_seqs - 1;
+        if (a.item_start[s_hint] <= k && k < a.item_start[s_hint + 1]) {
+            lo = hi = s_hint;
+        } else {
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (a.item_start[mid] <= k) lo = mid; else hi = mid - 1;
+            }
+        }
+        const int s = lo;
+        s_hint = s;
+        const int p = k - a.item_start[s];
+        const int L = a.seq_lens[s];
+        const int tok0 = p * a.split_tokens;
+        const int tok1 = min(L, tok0 + a.split_tokens);
+        const int nt = (tok1 - tok0 + kTileTok - 1) / kTileTok;
+
+        // q row for (s, h), 8 dims per lane, pre-scaled into log2 units
+        float qf[8];
+        {
+            const uint4 qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)s * a.H + h) * kD + 8 * li);
+            const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                qf[2 * c] = bf16lo(w[c]) * a.scale_log2;
+                qf[2 * c + 1] = bf16hi(w[c]) * a.scale_log2;
+            }
+        }
+
+        // prologue: fill the ring
+        if (lane == 0) {
+            for (int t = 0; t < nt && t < kStages; ++t) {
+                const int slot = (gtile + t) % kStages;
+                issue_tile(a, ring, slot, s, h, tok0 + t * kTileTok);
+                pending |= 1u << slot;
+            }
+        }
+        __syncwarp();
+
+        float m = -INFINITY, l = 0.f;
+        float o[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[c] = 0.f;
+
+        for (int t = 0; t < nt; ++t, ++gtile) {
+            const int slot = gtile % kStages;
+            const uint32_t parity = (gtile / kStages) & 1u;
+            if (!mbar_wait(ring.full + slot, parity, a.err)) { dead = true; break; }
+            if (lane == 0) pending &= ~(1u << slot);
+            const int tok = tok0 + t * kTileTok;
+            const bool tile_ok = resolve_block(a, s, tok) >= 0;
+            if (tile_ok) {
+                const uint8_t *kt = ring.slots + slot * kSlotBytes;
+                const uint8_t *vt = kt + kTileBytes;
+                float sc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 2 * i + half;
+                    const uint4 kv = *reinterpret_cast<const uint4 *>(kt + r * (kD * 2) + li * 16);
+                    const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+                    float acc = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        acc = fmaf(qf[2 * c], bf16lo(w[c]), acc);
+                        acc = fmaf(qf[2 * c + 1], bf16hi(w[c]), acc);
+                    }
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    sc[i] = (tok + r < tok1) ? acc : -INFINITY;
+                }
+                float mt = sc[0];
+#pragma unroll
+                for (int i = 1; i < 8; ++i) mt = fmaxf(mt, sc[i]);
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                const float m_new = fmaxf(m, mt);
+                const float alpha = ex2_approx(m - m_new);
+                float psum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    sc[i] = ex2_approx(sc[i] - m_new);
+                    psum += sc[i];
+                }
+                l = l * alpha + psum;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) o[c] *= alpha;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 2 * i + half;
+                    if (tok + r < tok1) {
+                        const uint4 vv = *reinterpret_cast<const uint4 *>(vt + r * (kD * 2) + li * 16);
+                        const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            o[2 * c] = fmaf(sc[i], bf16lo(w[c]), o[2 * c]);
+                            o[2 * c + 1] = fmaf(sc[i], bf16hi(w[c]), o[2 * c + 1]);
+                        }
+                    }
+                }
+                m = m_new;
+            }
+            __syncwarp();
+            if (lane == 0 && t + kStages < nt) {
+                issue_tile(a, ring, slot, s, h, tok + kStages * kTileTok);
+                pending |= 1u << slot;
+            }
+            __syncwarp();
+        }
+        if (dead) break;
+
+        // combine the two half-warps (same running max m)
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[c] += __shfl_xor_sync(0xffffffffu, o[c], 16);
+        const size_t pidx = ((size_t)s * a.H + h) * a.max_splits + p;
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        if (half == 0) {
+            float4 *dst = reinterpret_cast<float4 *>(a.part_o + pidx * kD + 8 * li);
+            dst[0] = make_float4(o[0] * inv_l, o[1] * inv_l, o[2] * inv_l, o[3] * inv_l);
+            dst[1] = make_float4(o[4] * inv_l, o[5] * inv_l, o[6] * inv_l, o[7] * inv_l);
+        }
+        if (lane == 0) a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
+    }
+
+    // after a timeout: wait (bounded) for this warp's copies still in flight
+    // so no bulk copy lands in shared memory after the CTA has exited
+    if (lane == 0 && pending) {
+        for (int i = 0; i < kStages; ++i) {
+            if (pending & (1u << i)) {
+                // the outstanding phase of slot i is the one after the last consumed
+                const uint32_t uses = gtile / kStages + ((uint32_t)i < gtile % kStages ? 1u : 0u);
+                mbar_wait(ring.full + i, uses & 1u, nullptr);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ merge
+
+__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
+    const int s = blockIdx.x;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int L = a.seq_lens[s];
+    bool bad = !seq_len_ok(L, a);
+    if (!bad) {
+        const int nb = (L + a.block_size - 1) / a.block_size;
+        int my_bad = 0;
+        for (int lb = threadIdx.x; lb < nb; lb += blockDim.x) {
+            const int phys = a.block_table[(size_t)s * a.max_blocks + lb];
+            my_bad |= (phys < 0 || phys >= a.num_blocks);
+        }
+        bad = __syncthreads_or(my_bad) != 0;
+    } else {
+        __syncthreads_or(0);
+    }
+    if (bad && threadIdx.x == 0 && a.err) {
+        atomicOr(a.err, seq_len_ok(L, a) ? ATTN_DEVERR_BLOCK_TABLE : ATTN_DEVERR_SEQ_LEN);
+    }
+    const int nsplit = bad ? 0 : (L + a.split_tokens - 1) / a.split_tokens;
+    for (int h = wid; h < a.H; h += blockDim.x / 32) {
+        const size_t base = ((size_t)s * a.H + h) * a.max_splits;
+        float M = -INFINITY;
+        for (int p = 0; p < nsplit; ++p) M = fmaxf(M, a.part_lse[base + p]);
+        float tot = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p = 0; p < nsplit; ++p) {
+            const float w = ex2_approx(a.part_lse[base + p] - M);
+            const float4 v = reinterpret_cast<const float4 *>(a.part_o + (base + p) * kD)[lane];
+            tot += w;
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        const float inv = tot > 0.f ? 1.f / tot : 0.f;
+        uint2 packed;
+        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2 *>(a.O + ((size_t)s * a.H + h) * kD + 4 * lane) = packed;
+        if (lane == 0)
+            a.LSE[(size_t)s * a.H + h] = tot > 0.f ? (M + __log2f(tot)) * 0.69314718055994530942f : -INFINITY;
+    }
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+    size_t counter, item_start, part_lse, part_o, total;
+};
+
+WsLayout ws_layout(int num_seqs, int H, int max_splits) {
+    WsLayout w;
+    w.counter = 0;
+    w.item_start = 256;
+    w.part_lse = align_up(w.item_start + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
+    w.part_o = align_up(w.part_lse + sizeof(float) * (size_t)num_seqs * H * max_splits, 256);
+    w.total = align_up(w.part_o + sizeof(float) * (size_t)num_seqs * H * max_splits * kD, 256);
+    return w;
+}
+
+}  // namespace
+
+int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_size) {
+    (void)d;
+    const long long max_len = (long long)max_blocks * block_size;
+    const long long work = (long long)num_seqs * H * max_len;
+    long long split = 256;
+    while (split < max_len && work / split > 65536) split <<= 1;
+    return (int)split;
+}
+
+int decode_max_splits(int num_seqs, int H, int d, int max_blocks, int block_size) {
+    const long long max_len = (long long)max_blocks * block_size;
+    const int split = decode_split_tokens(num_seqs, H, d, max_blocks, block_size);
+    return (int)((max_len + split - 1) / split);
+}
+
+size_t decode_workspace_bytes(int num_seqs, int H, int d, int max_blocks, int block_size) {
+    const int ms = decode_max_splits(num_seqs, H, d, max_blocks, block_size);
+    return ws_layout(num_seqs, H, ms < 1 ? 1 : ms).total;
+}
+
+attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
+    static int sm_count[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ECUDA;
+    if (dev < 0 || dev >= 64) return ATTN_ECUDA;
+    if (sm_count[dev] == 0) {
+        if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ATTN_ECUDA;
+        if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes) != cudaSuccess)
+            return ATTN_ECUDA;
+    }
+    DecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(p.q);
+    a.k_cache = static_cast<const __nv_bfloat16 *>(p.k_cache);
+    a.v_cache = static_cast<const __nv_bfloat16 *>(p.v_cache);
+    a.block_table = p.block_table;
+    a.seq_lens = p.seq_lens;
+    a.O = static_cast<__nv_bfloat16 *>(p.O);
+    a.LSE = p.LSE;
+    a.err = p.err_flag;
+    a.num_seqs = p.num_seqs;
+    a.H = p.H;
+    a.num_blocks = p.num_blocks;
+    a.max_blocks = p.max_blocks;
+    a.block_size = p.block_size;
+    a.split_tokens = decode_split_tokens(p.num_seqs, p.H, p.d, p.max_blocks, p.block_size);
+    a.max_splits = decode_max_splits(p.num_seqs, p.H, p.d, p.max_blocks, p.block_size);
+    if (a.max_splits < 1) a.max_splits = 1;
+    a.scale_log2 = p.scale * 1.4426950408889634f;
+    const WsLayout w = ws_layout(p.num_seqs, p.H, a.max_splits);
+    uint8_t *ws = static_cast<uint8_t *>(p.workspace);
+    a.counter = reinterpret_cast<int32_t *>(ws + w.counter);
+    a.item_start = reinterpret_cast<int32_t *>(ws + w.item_start);
+    a.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
+    a.part_o = reinterpret_cast<float *>(ws + w.part_o);
+
+    decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    decode_split_kernel<<<sm_count[dev], kWarps * 32, kSmemBytes, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    decode_merge_kernel<<<p.num_seqs, 128, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    return ATTN_OK;
+}
+
+}  // namespace osp

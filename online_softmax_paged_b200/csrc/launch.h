@@ -1,0 +1,42 @@
+// launch.h -- internal launcher interface between the C ABI (api.cu) and the
+// kernel translation units.  Not installed; the public ABI is include/attn.h.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/attn.h"
+
+namespace osp {
+
+struct DenseLaunch {
+    const void *Q, *K, *V;
+    void *O;
+    float *LSE;
+    int B, H, N, d, causal;
+    float scale;
+    int32_t *err_flag;
+};
+
+struct DecodeLaunch {
+    const void *q, *k_cache, *v_cache;
+    const int32_t *block_table, *seq_lens;
+    void *O;
+    float *LSE;
+    int num_seqs, H, d, num_blocks, max_blocks, block_size;
+    float scale;
+    void *workspace;
+    int32_t *err_flag;
+};
+
+attn_status launch_dense_f32(const DenseLaunch &p, cudaStream_t stream);
+attn_status launch_prefill_bf16(const DenseLaunch &p, cudaStream_t stream);
+attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream);
+
+int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_size);
+int decode_max_splits(int num_seqs, int H, int d, int max_blocks, int block_size);
+size_t decode_workspace_bytes(int num_seqs, int H, int d, int max_blocks, int block_size);
+
+}  // namespace osp

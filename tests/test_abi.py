@@ -1,0 +1,121 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/attn.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import online_softmax_paged_b200 as osp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_0-9]+)\s*\([^;{]*\)\s*;", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(osp.lib_path()):
+        from online_softmax_paged_b200 import build
+        build.build()
+    return osp.load()
+
+
+def test_header_declares_expected_functions():
+    assert _declared() == sorted(osp.EXPORTED_SYMBOLS)
+
+
+def test_every_declared_symbol_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", osp.lib_path()], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(_declared()) <= exported
+    # nothing else leaks: the kernels and helpers have hidden visibility
+    assert not any(s.startswith("_ZN3osp") for s in exported)
+
+
+def test_library_targets_sm100a_only():
+    out = subprocess.run(["cuobjdump", "--list-elf", osp.lib_path()], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}, archs
+
+
+FAKE = ctypes.c_void_p(4096)  # 16-byte aligned, never dereferenced: checks fail first
+
+
+def test_attn_fwd_rejects_on_host(lib):
+    f = lib.attn_fwd
+    ok_args = dict(B=1, H=2, N=8, d=128, causal=0, scale=0.125, dt=1)
+
+    def call(**kw):
+        a = {**ok_args, **kw}
+        ptrs = [kw.get(p, FAKE) for p in ("Q", "K", "V", "O", "LSE")]
+        return f(*ptrs, a["B"], a["H"], a["N"], a["d"], a["causal"], ctypes.c_float(a["scale"]), a["dt"], None, None)
+
+    assert call(Q=None) == osp.ATTN_EINVAL
+    assert call(N=0) == osp.ATTN_EINVAL
+    assert call(B=0) == osp.ATTN_EINVAL
+    assert call(scale=0.0) == osp.ATTN_EINVAL
+    assert call(scale=float("nan")) == osp.ATTN_EINVAL
+    assert call(dt=7) == osp.ATTN_EINVAL
+    assert call(d=96) == osp.ATTN_EUNSUPPORTED
+    assert call(d=256) == osp.ATTN_EUNSUPPORTED
+    assert call(Q=ctypes.c_void_p(4097)) == osp.ATTN_EINVAL
+
+
+def test_paged_decode_rejects_on_host(lib):
+    f = lib.paged_attn_decode
+    base = dict(block_size=16, S=2, H=4, d=128, nb=10, mb=4, scale=0.1, dt=1, ws=1 << 20)
+
+    def call(**kw):
+        a = {**base, **kw}
+        p = [kw.get(n, FAKE) for n in ("q", "k", "v", "bt", "sl")]
+        return f(*p, a["block_size"], kw.get("O", FAKE), kw.get("LSE", FAKE), a["S"], a["H"], a["d"], a["nb"],
+                 a["mb"], ctypes.c_float(a["scale"]), a["dt"], kw.get("w", FAKE), a["ws"], None, None)
+
+    assert call(q=None) == osp.ATTN_EINVAL
+    assert call(dt=0) == osp.ATTN_EUNSUPPORTED
+    assert call(d=64) == osp.ATTN_EUNSUPPORTED
+    assert call(block_size=8) == osp.ATTN_EUNSUPPORTED
+    assert call(block_size=64) == osp.ATTN_EUNSUPPORTED
+    assert call(nb=0) == osp.ATTN_EINVAL
+    assert call(scale=-1.0) == osp.ATTN_EINVAL
+    assert call(ws=16) == osp.ATTN_EINVAL
+    assert call(k=ctypes.c_void_p(4104)) == osp.ATTN_EINVAL
+    assert call(S=0) == osp.ATTN_OK  # nothing to do, nothing launched
+
+
+def test_workspace_size_and_split(lib):
+    ws = osp.paged_attn_decode_workspace_size(64, 32, 128, 256, 16)
+    st = osp.paged_attn_decode_split_tokens(64, 32, 128, 256, 16)
+    assert st >= 256 and st % 32 == 0
+    splits = -(-256 * 16 // st)
+    assert ws >= 64 * 32 * splits * (128 + 1) * 4
+    assert ws % 256 == 0
+    assert osp.paged_attn_decode_workspace_size(64, 32, 64, 256, 16) == 0
+    assert osp.paged_attn_decode_workspace_size(64, 0, 128, 256, 16) == 0
+    # the split size is a function of the sizes only
+    assert st == osp.paged_attn_decode_split_tokens(64, 32, 128, 256, 16)
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert osp.attn_status_str(s)
+    assert osp.attn_status_str(99) == "unknown status"
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        osp.attn_fwd(x, x, x)

@@ -1,0 +1,182 @@
+"""GPU parity of the paged decode entry point against the fp64 oracle.
+
+The oracle resolves every block table by explicit copy on the host; the
+kernel gathers through the table on the device.  Small workloads are checked
+in full (lengths 0, 1, 15, 16, 17, ..., max; block sizes 16 and 32); the two
+full-size decode workloads on sampled sequences; physical placement shuffles
+must give bit-identical output; bad tables and lengths set the device error
+bits and zero the affected sequence.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests._parity import check_close, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import online_softmax_paged_b200 as osp
+    osp.load()
+
+
+def _osp():
+    import online_softmax_paged_b200 as osp
+    return osp
+
+
+class DeviceCache:
+    """Host view of a device cache that copies one physical block on access."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, i):
+        return self.t[int(i)].float().cpu().numpy()
+
+
+def _decode(p, err=None, **kw):
+    O, LSE = _osp().paged_attn_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.block_size,
+                                      scale=p.scale, err_flag=err, **kw)
+    torch.cuda.synchronize()
+    return O, LSE
+
+
+def _oracle(p, seqs=None):
+    return oracle.paged_decode(to64(p.q), DeviceCache(p.k_cache), DeviceCache(p.v_cache), p.block_table.cpu().numpy(),
+                               p.seq_lens.cpu().numpy(), p.block_size, p.scale, seqs=seqs)
+
+
+EDGE_LENS = [0, 1, 2, 15, 16, 17, 31, 32, 33, 255, 256, 257, 511, 513, 1000, 2048]
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_edge_lengths_full(bs):
+    p = W.paged_uniform(H=32, d=128, block_size=bs, pool=600, len_hi=2048, seed=1, device="cuda", lens=EDGE_LENS)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _decode(p, err)
+    assert int(err.item()) == 0
+    O_ref, L_ref = _oracle(p)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"edge lens bs={bs}")
+    assert (O[0] == 0).all() and torch.isneginf(LSE[0]).all()  # seq_len 0
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_random_small_full(bs):
+    p = W.paged_uniform(num_seqs=23, H=8, d=128, block_size=bs, pool=3000, len_lo=1, len_hi=3000, seed=2,
+                        device="cuda")
+    O, LSE = _decode(p)
+    O_ref, L_ref = _oracle(p)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"random bs={bs}")
+
+
+def test_placement_shuffle_bit_identical_small():
+    p = W.paged_uniform(num_seqs=11, H=4, d=128, block_size=16, pool=2000, len_lo=1, len_hi=3000, seed=3,
+                        device="cuda")
+    O1, L1 = _decode(p)
+    for seed in (1, 2):
+        O2, L2 = _decode(W.shuffle_placement(p, seed=seed))
+        assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+def test_decode_uniform_full_size():
+    """64 sequences, H=32, d=128, bs=16, lengths U[128, 4096], pool 20000,
+    seed 0: eight sampled sequences (shortest, longest and six others) in
+    full against the oracle; all sequences for finiteness; a placement
+    shuffle of the whole pool is bit-identical."""
+    p = W.paged_uniform(device="cuda", seed=0, **W.DECODE_UNIFORM)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _decode(p, err)
+    assert int(err.item()) == 0
+    assert torch.isfinite(O.float()).all() and torch.isfinite(LSE).all()
+    sl = p.seq_lens.cpu().numpy()
+    seqs = sorted({int(sl.argmin()), int(sl.argmax()), 0, 9, 21, 33, 47, 63})
+    O_ref, L_ref = _oracle(p, seqs=seqs)
+    check_close(O[seqs], LSE[seqs], O_ref[seqs], L_ref[seqs], torch.bfloat16, "decode uniform")
+    O2, L2 = _decode(W.shuffle_placement(p, seed=11))
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
+
+
+def test_decode_shared_prefix_full_size():
+    """256 sequences, bs=32, log-normal lengths, 8-sequence groups sharing a
+    512-token prefix, seed 0: two whole groups in full against the oracle."""
+    p = W.paged_shared_prefix(device="cuda", seed=0, **W.DECODE_SHARED_PREFIX)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _decode(p, err)
+    assert int(err.item()) == 0
+    assert torch.isfinite(O.float()).all() and torch.isfinite(LSE).all()
+    seqs = p.shared_groups[0] + p.shared_groups[17]
+    O_ref, L_ref = _oracle(p, seqs=seqs)
+    check_close(O[seqs], LSE[seqs], O_ref[seqs], L_ref[seqs], torch.bfloat16, "decode shared prefix")
+
+
+def test_bad_block_table_entry_flags_and_zeroes():
+    osp = _osp()
+    p = W.paged_uniform(num_seqs=6, H=4, d=128, block_size=16, pool=900, len_lo=100, len_hi=1500, seed=4,
+                        device="cuda")
+    t = p.block_table.clone()
+    t[2, 3] = p.num_blocks + 5
+    t[4, 0] = -7
+    bad = W.PagedInputs(p.q, p.k_cache, p.v_cache, t, p.seq_lens, p.block_size, p.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _decode(bad, err)
+    assert osp.attn_read_error(err) & osp.ATTN_DEVERR_BLOCK_TABLE
+    for s in (2, 4):
+        assert (O[s] == 0).all() and torch.isneginf(LSE[s]).all()
+    good = [0, 1, 3, 5]
+    O_ref, L_ref = _oracle(p, seqs=good)
+    check_close(O[good], LSE[good], O_ref[good], L_ref[good], torch.bfloat16, "good rows beside bad ones")
+
+
+def test_bad_seq_len_flags_and_zeroes():
+    osp = _osp()
+    p = W.paged_uniform(num_seqs=4, H=4, d=128, block_size=16, pool=500, len_lo=10, len_hi=400, seed=5,
+                        device="cuda")
+    sl = p.seq_lens.clone()
+    sl[1] = p.max_blocks_per_seq * 16 + 1
+    sl[3] = -2
+    bad = W.PagedInputs(p.q, p.k_cache, p.v_cache, p.block_table, sl, p.block_size, p.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _decode(bad, err)
+    assert osp.attn_read_error(err) & osp.ATTN_DEVERR_SEQ_LEN
+    for s in (1, 3):
+        assert (O[s] == 0).all() and torch.isneginf(LSE[s]).all()
+    O_ref, L_ref = _oracle(p, seqs=[0, 2])
+    check_close(O[[0, 2]], LSE[[0, 2]], O_ref[[0, 2]], L_ref[[0, 2]], torch.bfloat16, "good rows")
+
+
+def test_workspace_too_small_rejected():
+    osp = _osp()
+    p = W.paged_uniform(num_seqs=3, H=4, d=128, block_size=16, pool=300, len_lo=10, len_hi=400, seed=6,
+                        device="cuda")
+    ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(osp.AttnError):
+        _decode(p, workspace=ws)
+
+
+def test_decode_equals_dense_last_row():
+    """Paging changes storage, not the math: with an identity table the decode
+    of the last token equals the dense causal prefill's last row (both within
+    tolerance of the same oracle value)."""
+    osp = _osp()
+    H, d, bs, L = 4, 128, 16, 700
+    nb = -(-L // bs)
+    dense = W.dense_inputs(1, H, nb * bs, d, dtype=torch.bfloat16, seed=9, device="cuda", causal=True)
+    kc = dense["K"][0].view(H, nb, bs, d).permute(1, 0, 2, 3).contiguous()
+    vc = dense["V"][0].view(H, nb, bs, d).permute(1, 0, 2, 3).contiguous()
+    q = dense["Q"][0, :, L - 1].contiguous().view(1, H, d)
+    table = torch.arange(nb, dtype=torch.int32, device="cuda").view(1, nb)
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    O, LSE = osp.paged_attn_decode(q, kc, vc, table, sl, bs)
+    Od, Ld = osp.attn_fwd(dense["Q"][:, :, :L].contiguous(), dense["K"][:, :, :L].contiguous(),
+                          dense["V"][:, :, :L].contiguous(), causal=True)
+    torch.cuda.synchronize()
+    assert (O[0].float() - Od[0, :, L - 1].float()).abs().max().item() <= 2e-2
+    assert (LSE[0] - Ld[0, :, L - 1]).abs().max().item() <= 1e-3

@@ -108,16 +108,21 @@ def _cache(pool, H, bs, d, g, device, dtype):
 
 
 def paged_uniform(num_seqs=64, H=32, d=128, block_size=16, pool=20000, len_lo=128, len_hi=4096,
-                  seed=0, device="cpu", dtype=torch.bfloat16, max_blocks_per_seq=None):
+                  seed=0, device="cpu", dtype=torch.bfloat16, max_blocks_per_seq=None, lens=None):
     """Paged decode workload with independent random placement.
 
     Draw order: seq_lens ~ U{len_lo..len_hi}; one randperm(pool), sliced
     consecutively into each sequence's ceil(L / block_size) blocks (so no
     physical block is used twice, within or across sequences); K cache;
-    V cache; q.  Unused block-table entries are -1.
+    V cache; q.  Unused block-table entries are -1.  ``lens`` replaces the
+    length draw with given lengths (edge-case tests).
     """
     g = _gen(seed, device)
-    seq_lens = torch.randint(len_lo, len_hi + 1, (num_seqs,), generator=g, device=device)
+    if lens is not None:
+        seq_lens = torch.tensor(list(lens), dtype=torch.int64, device=device)
+        num_seqs = len(lens)
+    else:
+        seq_lens = torch.randint(len_lo, len_hi + 1, (num_seqs,), generator=g, device=device)
     perm = torch.randperm(pool, generator=g, device=device)
     seq_lens_c = seq_lens.cpu()
     perm_c = perm.cpu()
