@@ -95,7 +95,9 @@ def barrier(ws: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while timing."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms from the
+    warm-up through the timed region (the soak keeps the GPU loaded for a
+    while first, so short timed regions still have loaded samples)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -110,7 +112,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
             time.sleep(0.25)
@@ -120,7 +122,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -131,10 +133,14 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and the throttle reasons seen between t0 and t1
+        (perf_counter seconds; default: every sample)."""
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for t, line in self.lines:
+            if (t0 is not None and t < t0) or (t1 is not None and t > t1 + 0.15):
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -256,11 +262,16 @@ class Decode:
         self.name = name
         if name == "decode_uniform":
             self.p = W.paged_uniform(device=device, seed=seed, **W.DECODE_UNIFORM)
+        elif name == "decode_uniform_small":
+            # 16 sequences of the uniform workload in a 4000-block pool (1 GiB
+            # of K/V, still above L2): the case profiler captures run on
+            self.p = W.paged_uniform(device=device, seed=seed, **{**W.DECODE_UNIFORM, "num_seqs": 16,
+                                                                   "pool": 4000})
         else:
             self.p = W.paged_shared_prefix(device=device, seed=seed, **W.DECODE_SHARED_PREFIX)
         self.logical = W.logical_kv_bytes(self.p)
         self.unique = W.unique_kv_bytes(self.p)
-        self.work = float(self.unique if name != "decode_uniform" else self.logical)  # bytes per step
+        self.work = float(self.unique if name == "decode_shared_prefix" else self.logical)  # bytes per step
         self.O = torch.empty_like(self.p.q)
         self.LSE = torch.empty(self.p.q.shape[:2], dtype=torch.float32, device=device)
         import online_softmax_paged_b200 as osp
@@ -350,18 +361,28 @@ def make_workload(name, device, seed=0):
         return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
     if name == "prefill_16k":
         return Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
-    if name in ("decode_uniform", "decode_shared_prefix"):
+    if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small"):
         return Decode(name, device, seed)
     raise SystemExit(f"unknown workload {name}")
 
 
 # ---------------------------------------------------------------- timing
 
-def time_steps(wl, osp, steps, warmup, device, ws):
+def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0):
+    """W warm-up steps, an optional untimed soak (so the clocks sampled
+    around the timed region reflect a loaded GPU), then K timed steps between
+    barrier + synchronize with CUDA events around every launch."""
     st = torch.cuda.current_stream(device)
     for i in range(warmup):
         wl.step(i, osp)
     torch.cuda.synchronize(device)
+    if soak_s > 0:
+        t0, i = time.perf_counter(), 0
+        while time.perf_counter() - t0 < soak_s:
+            for _ in range(8):
+                wl.step(i, osp)
+                i += 1
+            torch.cuda.synchronize(device)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(ws)
     torch.cuda.synchronize(device)
@@ -412,7 +433,9 @@ def run_ours(args):
     wl = make_workload(args.workload, device, seed=args.seed + rank)
     bound = "tensor" if isinstance(wl, Prefill) else "hbm"
     with ClockSampler(local) as clocks:
-        per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws)
+        t_load0 = time.perf_counter()
+        per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak)
+        t_load1 = time.perf_counter()
     t_max = max_over_ranks(total_ms, ws)
     work_all = sum_over_ranks(wl.work * args.steps, ws)
     value = work_all / (t_max * 1e-3) / wl.scale_unit
@@ -425,7 +448,7 @@ def run_ours(args):
     extra = {}
     if args.workload == "prefill_2k" and not args.no_decode:
         dec = make_workload("decode_uniform", device, seed=args.seed + rank)
-        per_d, total_d, _ = time_steps(dec, osp, args.steps, args.warmup, device, ws)
+        per_d, total_d, _ = time_steps(dec, osp, args.steps, args.warmup, device, ws, soak_s=min(args.soak, 0.5))
         td = max_over_ranks(total_d, ws)
         extra["decode"] = {"workload": "decode_uniform", "value": round(sum_over_ranks(dec.work * args.steps, ws)
                                                                         / (td * 1e-3) / 1e9, 2),
@@ -448,7 +471,7 @@ def run_ours(args):
                 "roofline": rl, "cpu_baseline": cpu,
                 "e2e": {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-                "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks.summary(),
+                "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks.summary(t_load0, t_load1),
                 "timed_wall_s": round(wall, 3), **extra}
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -546,11 +569,13 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_2k",
-                    choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix"])
+                    choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
+                             "decode_uniform_small"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode leg of the default line")
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing (clocks)")
     args = ap.parse_args(argv)
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
