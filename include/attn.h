@@ -140,6 +140,37 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
                               int32_t *err_flag, attn_stream_t stream);
 
 /*
+ * Paged decode without a workspace argument, for callers that cannot
+ * allocate device memory (code running where cudaMalloc is not permitted or
+ * not wanted, e.g. inside an allocator or pool callback, in a process whose
+ * device memory is fixed up front, or a plain C program with no framework to
+ * borrow memory from).  The pages have no counterpart: this is a deployment
+ * convenience, not part of the method.
+ *
+ * Arguments, layouts, results and device checks are those of
+ * paged_attn_decode.  The split-KV scratch is a fixed array of
+ * ATTN_NOALLOC_SCRATCH_BYTES compiled into the library, reserved on every GPU
+ * that loads the library for the life of the process; the call itself
+ * allocates nothing.
+ *   - Sizes whose workspace (paged_attn_decode_workspace_size) exceeds
+ *     ATTN_NOALLOC_SCRATCH_BYTES return ATTN_EUNSUPPORTED, nothing launched.
+ *   - Every call on a device shares the one scratch array: calls whose
+ *     kernels can overlap on the GPU (streams without ordering between them)
+ *     race and give wrong results.  Calls on one stream are safe.
+ *   - The scratch keeps the previous call's contents; whatever must start at
+ *     zero is cleared by the call itself.
+ *   - The first call made while a device is current looks up the scratch
+ *     address with a runtime call; make that first call before any stream
+ *     capture starts.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+ATTN_API attn_status paged_attn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                      const int32_t *block_table, const int32_t *seq_lens, int block_size,
+                                      void *O, float *LSE,
+                                      int num_seqs, int H, int d, int num_blocks, int max_blocks_per_seq,
+                                      float scale, attn_dtype dt, int32_t *err_flag, attn_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device int32 at err_flag and return
  * ATTN_OK if it is 0, ATTN_EDEVICE otherwise (the bits are written to
  * *bits_out when it is not NULL).  The flag is not reset.

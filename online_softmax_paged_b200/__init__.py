@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "AttnError", "attn_fwd", "paged_attn_decode", "paged_attn_decode_workspace_size",
-    "paged_attn_decode_split_tokens", "attn_read_error", "attn_status_str", "lib_path", "load",
+    "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "EXPORTED_SYMBOLS",
 ]
 
@@ -28,7 +28,10 @@ ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT = 1, 2, 4
 
 # every function include/attn.h declares
 EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
-                    "paged_attn_decode", "attn_read_error", "attn_status_str")
+                    "paged_attn_decode", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str")
+
+# size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
+ATTN_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -62,6 +65,9 @@ def load():
     lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                       c_float, c_int, vp, c_size, vp, vp]
     lib.paged_attn_decode.restype = c_int
+    lib.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
+                                              c_float, c_int, vp, vp]
+    lib.paged_attn_decode_noalloc.restype = c_int
     lib.attn_read_error.argtypes = [vp, i32p, vp]
     lib.attn_read_error.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
@@ -162,6 +168,41 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=
                                   _ptr(err_flag), _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode")
+    return O, LSE
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, block_size, O=None, LSE=None,
+                              scale=None, err_flag=None, stream=None):
+    """Paged decode that passes no workspace: the library uses its own fixed
+    scratch array (ATTN_NOALLOC_SCRATCH_BYTES), for callers that cannot
+    allocate device memory.  Calls that may overlap on the GPU share that
+    scratch and race; keep them on one stream.  The first call on a device
+    looks up the scratch address, so make it before any graph capture.
+    O and LSE are allocated here when not given (pass them to allocate
+    nothing).  Raises AttnError (ATTN_EUNSUPPORTED) when the sizes need more
+    scratch than the array holds."""
+    _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, err_flag)
+    S, H, d = q.shape
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if k_cache.shape != v_cache.shape or k_cache.shape[1] != H or k_cache.shape[2] != block_size or \
+            k_cache.shape[3] != d:
+        raise ValueError("caches must be [num_blocks, H, block_size, d]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((S, H), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = load().paged_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                          _ptr(seq_lens), int(block_size), _ptr(O), _ptr(LSE), S, H, d,
+                                          k_cache.shape[0], block_table.shape[1], float(scale),
+                                          _dtype_code(q.dtype), _ptr(err_flag), _stream(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_attn_decode_noalloc (scratch limit %d bytes)" % ATTN_NOALLOC_SCRATCH_BYTES)
     return O, LSE
 
 
