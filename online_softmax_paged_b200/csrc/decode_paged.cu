@@ -10,25 +10,30 @@
 // tokens, contiguous logical / non-contiguous physical blocks.
 //
 // B200 design (HBM-bound: ~1 flop per byte):
-//   1. plan kernel      -- one CTA scans seq_lens into per-sequence split
-//                          offsets (split size fixed by the host from the
-//                          sizes only) and zeroes the work counter.
-//   2. split kernel     -- persistent, one CTA per SM, every warp an
-//                          independent worker.  A warp takes (sequence, split,
-//                          head) items from an atomic counter and streams the
-//                          split's 16-token K and V tiles (4 KiB each,
-//                          contiguous inside a block) into its own ring of
-//                          shared-memory slots with 1-D bulk async copies
-//                          completing on per-slot mbarriers.  Math reads the
-//                          slots with 16-byte vector loads: a half-warp holds
-//                          one 128-wide row (8 dims per lane), q.k is reduced
-//                          with warp shuffles, and the online-softmax update is
-//                          applied once per tile.  Each item writes a
-//                          normalised partial O and its log2-sum-exp.
-//   3. merge kernel     -- per sequence: validate the table, then
-//                          LSE = log sum_p exp(LSE_p), O = sum_p e^{LSE_p-LSE} O_p.
-// Every arithmetic order depends only on logical token positions, so moving
-// blocks to other physical ids gives bit-identical results.
+//   1. plan kernel  -- one CTA scans seq_lens into per-sequence split offsets
+//                      (split size fixed by the host from the sizes only),
+//                      zeroes the work counter and the per-(sequence, head)
+//                      completion counters, and writes the result of empty or
+//                      invalid-length sequences (O = 0, LSE = -inf).
+//   2. split kernel -- persistent, one CTA per SM, every warp an independent
+//                      worker, launched as a programmatic dependent of the
+//                      plan.  A warp takes (sequence, split, head) items from
+//                      an atomic counter and streams the split's 16-token K
+//                      and V tiles (4 KiB each, contiguous inside a block)
+//                      into its own ring of shared-memory slots with 1-D bulk
+//                      async copies completing on per-slot mbarriers.  Math
+//                      reads the slots with 16-byte vector loads: a half-warp
+//                      holds one 128-wide row (8 dims per lane), q.k is reduced
+//                      with warp shuffles, and the online-softmax update is
+//                      applied once per tile.  A sequence with one split
+//                      writes O and LSE directly; otherwise each split writes
+//                      a normalised partial O and its log2-sum-exp, and the
+//                      warp that completes the last split of a (sequence,
+//                      head) merges them in split order:
+//                      LSE = log sum_p exp(LSE_p), O = sum_p e^{LSE_p-LSE} O_p.
+// Every arithmetic order depends only on logical token positions (which warp
+// runs a split, or merges, changes nothing), so moving blocks to other
+// physical ids gives bit-identical results.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -60,6 +65,8 @@ struct DecodeArgs {
     // workspace views
     int32_t *counter;     // [1]
     int32_t *item_start;  // [num_seqs + 1] prefix sum of splits per sequence
+    int32_t *done_cnt;    // [num_seqs, H] splits finished per (sequence, head)
+    int32_t *seq_bad;     // [num_seqs] nonzero: a block-table entry was out of range
     float *part_lse;      // [num_seqs, H, max_splits] log2 units
     float *part_o;        // [num_seqs, H, max_splits, d] normalised
     int num_seqs, H, num_blocks, max_blocks, block_size, split_tokens, max_splits;
@@ -72,13 +79,32 @@ __device__ __forceinline__ bool seq_len_ok(int L, const DecodeArgs &a) {
 
 // ------------------------------------------------------------------ plan
 
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    pdl_launch_dependents();  // the split kernel may start its prologue now
     if (tid == 0) {
         carry = 0;
         *a.counter = 0;
+    }
+    for (int i = tid; i < a.num_seqs * a.H; i += 1024) a.done_cnt[i] = 0;
+    for (int i = tid; i < a.num_seqs; i += 1024) a.seq_bad[i] = 0;
+    // sequences with no split: empty (L = 0) or an invalid length
+    for (int i = tid; i < a.num_seqs * a.H * (kD / 8); i += 1024) {
+        const int sh = i / (kD / 8), s = sh / a.H;
+        const int L = a.seq_lens[s];
+        if (L > 0 && seq_len_ok(L, a)) continue;
+        const int c = i % (kD / 8);
+        reinterpret_cast<uint4 *>(a.O + (size_t)sh * kD)[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (c == 0) a.LSE[sh] = -INFINITY;
+        if (c == 0 && (sh % a.H) == 0 && !seq_len_ok(L, a) && a.err) atomicOr(a.err, ATTN_DEVERR_SEQ_LEN);
     }
     __syncthreads();
     for (int base = 0; base < a.num_seqs; base += 1024) {
@@ -153,6 +179,25 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const WarpRing &
     bulk_g2s(dst + kTileBytes, a.v_cache + off, kTileBytes, bar);
 }
 
+constexpr float kLn2 = 0.69314718055994530942f;
+
+// Final bf16 row of O (o * inv_l, or zeros when o is null) and its LSE.
+// Lanes of half 0 hold dims 8*li .. 8*li+7.
+__device__ __forceinline__ void inv_l_store(const DecodeArgs &a, size_t sh, int li, int half, int lane,
+                                            const float *o, float inv_l, float lse) {
+    if (half == 0) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (o) {
+            w.x = pack_bf16x2(o[0] * inv_l, o[1] * inv_l);
+            w.y = pack_bf16x2(o[2] * inv_l, o[3] * inv_l);
+            w.z = pack_bf16x2(o[4] * inv_l, o[5] * inv_l);
+            w.w = pack_bf16x2(o[6] * inv_l, o[7] * inv_l);
+        }
+        *reinterpret_cast<uint4 *>(a.O + sh * kD + 8 * li) = w;
+    }
+    if (lane == 0) a.LSE[sh] = lse;
+}
+
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -166,6 +211,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     __syncwarp();
 
     const int half = lane >> 4, li = lane & 15;
+    pdl_wait();  // the plan kernel's writes are visible from here on
     const int total = a.item_start[a.num_seqs] * a.H;
     uint32_t gtile = 0;  // tiles consumed by this warp so far (ring phase)
     uint32_t pending = 0;  // lane 0: slots with a copy in flight
@@ -222,6 +268,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         float o[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) o[c] = 0.f;
+        bool saw_bad = false;
 
         for (int t = 0; t < nt; ++t, ++gtile) {
             const int slot = gtile % kStages;
@@ -230,6 +277,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             if (lane == 0) pending &= ~(1u << slot);
             const int tok = tok0 + t * kTileTok;
             const bool tile_ok = resolve_block(a, s, tok) >= 0;
+            saw_bad |= !tile_ok;
             if (tile_ok) {
                 const uint8_t *kt = ring.slots + slot * kSlotBytes;
                 const uint8_t *vt = kt + kTileBytes;
@@ -294,14 +342,60 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         l += __shfl_xor_sync(0xffffffffu, l, 16);
 #pragma unroll
         for (int c = 0; c < 8; ++c) o[c] += __shfl_xor_sync(0xffffffffu, o[c], 16);
-        const size_t pidx = ((size_t)s * a.H + h) * a.max_splits + p;
+        const int nsplit = a.item_start[s + 1] - a.item_start[s];
+        const size_t sh = (size_t)s * a.H + h;
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        if (nsplit == 1) {
+            // whole sequence in this item: final result, no partial round trip
+            if (saw_bad) {
+                inv_l_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
+            } else {
+                inv_l_store(a, sh, li, half, lane, o, inv_l, l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY);
+            }
+            continue;
+        }
+        const size_t pidx = sh * a.max_splits + p;
         if (half == 0) {
             float4 *dst = reinterpret_cast<float4 *>(a.part_o + pidx * kD + 8 * li);
             dst[0] = make_float4(o[0] * inv_l, o[1] * inv_l, o[2] * inv_l, o[3] * inv_l);
             dst[1] = make_float4(o[4] * inv_l, o[5] * inv_l, o[6] * inv_l, o[7] * inv_l);
         }
-        if (lane == 0) a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
+        if (lane == 0) {
+            a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
+            if (saw_bad) atomicOr(a.seq_bad + s, 1);
+        }
+        __threadfence();  // partials (and the bad mark) before the completion count
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(a.done_cnt + sh, 1) == nsplit - 1);
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        // this warp finished the last split of (s, h): merge in split order
+        __threadfence();
+        if (__ldcg(a.seq_bad + s)) {
+            inv_l_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
+            continue;
+        }
+        const float *plse = a.part_lse + sh * a.max_splits;
+        float M = -INFINITY;
+        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(plse + q));
+        float tot = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < nsplit; ++q) {
+            const float w = ex2_approx(__ldcg(plse + q) - M);
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sh * a.max_splits + q) * kD) + lane);
+            tot += w;
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        const float inv = tot > 0.f ? 1.f / tot : 0.f;
+        uint2 packed;
+        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = packed;
+        if (lane == 0) a.LSE[sh] = tot > 0.f ? (M + __log2f(tot)) * kLn2 : -INFINITY;
     }
 
     // after a timeout: wait (bounded) for this warp's copies still in flight
@@ -317,64 +411,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     }
 }
 
-// ------------------------------------------------------------------ merge
-
-__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
-    const int s = blockIdx.x;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int L = a.seq_lens[s];
-    bool bad = !seq_len_ok(L, a);
-    if (!bad) {
-        const int nb = (L + a.block_size - 1) / a.block_size;
-        int my_bad = 0;
-        for (int lb = threadIdx.x; lb < nb; lb += blockDim.x) {
-            const int phys = a.block_table[(size_t)s * a.max_blocks + lb];
-            my_bad |= (phys < 0 || phys >= a.num_blocks);
-        }
-        bad = __syncthreads_or(my_bad) != 0;
-    } else {
-        __syncthreads_or(0);
-    }
-    if (bad && threadIdx.x == 0 && a.err) {
-        atomicOr(a.err, seq_len_ok(L, a) ? ATTN_DEVERR_BLOCK_TABLE : ATTN_DEVERR_SEQ_LEN);
-    }
-    const int nsplit = bad ? 0 : (L + a.split_tokens - 1) / a.split_tokens;
-    for (int h = wid; h < a.H; h += blockDim.x / 32) {
-        const size_t base = ((size_t)s * a.H + h) * a.max_splits;
-        float M = -INFINITY;
-        for (int p = 0; p < nsplit; ++p) M = fmaxf(M, a.part_lse[base + p]);
-        float tot = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = 0; p < nsplit; ++p) {
-            const float w = ex2_approx(a.part_lse[base + p] - M);
-            const float4 v = reinterpret_cast<const float4 *>(a.part_o + (base + p) * kD)[lane];
-            tot += w;
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
-        const float inv = tot > 0.f ? 1.f / tot : 0.f;
-        uint2 packed;
-        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2 *>(a.O + ((size_t)s * a.H + h) * kD + 4 * lane) = packed;
-        if (lane == 0)
-            a.LSE[(size_t)s * a.H + h] = tot > 0.f ? (M + __log2f(tot)) * 0.69314718055994530942f : -INFINITY;
-    }
-}
-
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t counter, item_start, part_lse, part_o, total;
+    size_t counter, item_start, done_cnt, seq_bad, part_lse, part_o, total;
 };
 
 WsLayout ws_layout(int num_seqs, int H, int max_splits) {
     WsLayout w;
     w.counter = 0;
     w.item_start = 256;
-    w.part_lse = align_up(w.item_start + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
+    w.done_cnt = align_up(w.item_start + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
+    w.seq_bad = align_up(w.done_cnt + sizeof(int32_t) * (size_t)num_seqs * H, 256);
+    w.part_lse = align_up(w.seq_bad + sizeof(int32_t) * (size_t)num_seqs, 256);
     w.part_o = align_up(w.part_lse + sizeof(float) * (size_t)num_seqs * H * max_splits, 256);
     w.total = align_up(w.part_o + sizeof(float) * (size_t)num_seqs * H * max_splits * kD, 256);
     return w;
@@ -436,15 +485,26 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     uint8_t *ws = static_cast<uint8_t *>(p.workspace);
     a.counter = reinterpret_cast<int32_t *>(ws + w.counter);
     a.item_start = reinterpret_cast<int32_t *>(ws + w.item_start);
+    a.done_cnt = reinterpret_cast<int32_t *>(ws + w.done_cnt);
+    a.seq_bad = reinterpret_cast<int32_t *>(ws + w.seq_bad);
     a.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
     a.part_o = reinterpret_cast<float *>(ws + w.part_o);
 
     decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-    decode_split_kernel<<<sm_count[dev], kWarps * 32, kSmemBytes, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-    decode_merge_kernel<<<p.num_seqs, 128, 0, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    // the split kernel is a programmatic dependent of the plan: its launch and
+    // barrier set-up overlap the plan; griddepcontrol.wait orders the data
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sm_count[dev]);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_split_kernel, a) != cudaSuccess) return ATTN_ECUDA;
     return ATTN_OK;
 }
 

@@ -111,6 +111,98 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
     }
 }
 
+
+// ---------------------------------------------------------------- softmax math
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe, keeping the MUFU free for the
+// rest.  Range reduction x = n + f with n = round(x) (the 1.5 * 2^23 shift),
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted to 2^f on [-1/2, 1/2]
+// at Chebyshev nodes with relative-error weighting (Lawson iterations towards
+// the minimax fit; max relative error 7.5e-5 in fp32, far below the bf16
+// rounding of P); 2^n is added into the exponent field.  x is clamped to
+// >= -125 so the result stays a normal number (2^-125 ~ 0 next to l >= 1).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0x1.fff692p-1f, c1 = 0x1.62f31ap-1f, c2 = 0x1.f0de1ap-3f, c3 = 0x1.c3f75ep-5f;
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    const uint64_t xc = f2_pack(x0, x1);
+    const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));           // n in the low mantissa bits
+    const uint64_t nr = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(kShift, kShift));  // -n
+    const uint64_t fr = f2_add(xc, nr);                               // f = x - n
+    uint64_t r = f2_fma(f2_pack(c3, c3), fr, f2_pack(c2, c2));
+    r = f2_fma(r, fr, f2_pack(c1, c1));
+    r = f2_fma(r, fr, f2_pack(c0, c0));
+    float p0, p1, t0, t1;
+    f2_unpack(r, p0, p1);
+    f2_unpack(t, t0, t1);
+    p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return f2_pack(p0, p1);
+}
+
+// Pairs k with (k % 8) >= kPolyFrom take the polynomial; the others MUFU ex2.
+constexpr int kPolyFrom = 5;  // 3 of every 8 pairs
+
+// P = 2^(s * scale_log2 - m) for one 128-wide score row held as raw fp32 bits
+// in sr, packed to bf16 pairs and stored over the first 64 TMEM columns of
+// the row's S region; the fp32 values are summed into acc2 (4 pairs of
+// accumulators).  USE_POLY sends 3 of every 8 pairs to the FMA-pipe
+// polynomial (only for tiles without masked entries).
+template <bool USE_POLY>
+__device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint32_t s_tm, uint64_t scale2,
+                                               uint64_t negm2, uint64_t (&acc2)[4]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int c = 2 * h + (e >> 4), k = (e & 15) * 2;
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sr[c][k]), __uint_as_float(sr[c][k + 1])), scale2, negm2);
+            uint64_t p2;
+            if (USE_POLY && (e & 7) >= kPolyFrom) {
+                p2 = exp2_poly2(x2);
+            } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            acc2[e & 3] = f2_add(acc2[e & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_tm + 32 * h, pk);
+    }
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -291,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_tm = tmem + lane_off + 2 * BN + i * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nkv[i]; ++j) {
+        const int my_nkv = i ? nkv[1] : nkv[0];
+        for (int j = 0; j < my_nkv; ++j) {
             ok = wait_or_abort(&s_full[i], j & 1, a.err, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -299,39 +392,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + 32 * c, sr[c]);
             tmem_wait_ld();
-            // visible keys: col <= lim (causal diagonal tile / sequence tail)
-            int lim = BN - 1;
-            if (CAUSAL && j == qt) lim = r;
-            lim = min(lim, a.N - 1 - j * BN);
-            float mx = -INFINITY;
+            // visible keys: col <= lim; only the causal diagonal tile and the
+            // sequence's last tile need masking
+            const bool masked = (CAUSAL && j == qt) || ((j + 1) * BN > a.N);
+            if (masked) {
+                int lim = BN - 1;
+                if (CAUSAL && j == qt) lim = r;
+                lim = min(lim, a.N - 1 - j * BN);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+            }
+            float mxa[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mxa[k] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float x = __uint_as_float(sr[c][e]);
-                    if (32 * c + e > lim) x = -INFINITY;
-                    sr[c][e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                for (int e = 0; e < 32; e += 8) {
+                    const int k = (e >> 3) + 4 * (c & 1);
+                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
+                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 4]), __uint_as_float(sr[c][e + 5]));
+                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 6]), __uint_as_float(sr[c][e + 7]));
                 }
+            const float mx = max3(max3(mxa[0], mxa[1], mxa[2]), max3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
             const float mx2 = mx * a.scale_log2;
             float m_ref = m;
             if (mx2 > m + kRescaleThreshold) m_ref = mx2;
             if (m_ref == -INFINITY) m_ref = 0.f;  // row with nothing visible yet
             const float alpha = ex2_approx(m - m_ref);
-            const float neg = -m_ref;
-            float psum = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = 2 * h + (e >> 4), k = (e & 15) * 2;
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][k]), a.scale_log2, neg));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][k + 1]), a.scale_log2, neg));
-                    psum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
-                tmem_st32(s_tm + 32 * h, pk);
+            const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
+            const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+            uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+            if (masked)
+                exp_pack_store<false>(sr, s_tm, scale2, negm2, acc2);
+            else
+                exp_pack_store<true>(sr, s_tm, scale2, negm2, acc2);
+            float psum;
+            {
+                const uint64_t t2 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+                float u0, u1;
+                f2_unpack(t2, u0, u1);
+                psum = u0 + u1;
             }
             l = l * alpha + psum;
             const bool need = (m_ref != m) && j > 0;
@@ -355,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&p_full[i]);
         }
-        if (ok && nkv[i] > 0) {
-            ok = wait_or_abort(&o_full[i], (nkv[i] - 1) & 1, a.err, abort_flag);
+        if (ok && my_nkv > 0) {
+            ok = wait_or_abort(&o_full[i], (my_nkv - 1) & 1, a.err, abort_flag);
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
