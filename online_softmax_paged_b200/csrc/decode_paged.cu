@@ -48,10 +48,11 @@ namespace {
 constexpr int kD = 128;                         // head dim supported here
 constexpr int kTileTok = 16;                    // tokens per pipeline tile
 constexpr int kTileBytes = kTileTok * kD * 2;   // 4 KiB of K (or of V)
-constexpr int kWarps = 8;                       // workers per CTA
-constexpr int kStages = 3;                      // ring slots per worker
+constexpr int kWarps = 12;                      // workers per CTA
+constexpr int kStages = 2;                      // ring slots per worker
 constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
-constexpr int kSmemBytes = kWarps * kStages * kSlotBytes + kWarps * kStages * 8 + 64;
+constexpr int kMaxSmemSeqs = 4096;  // split offsets staged in shared memory up to this many sequences
+constexpr int kSmemBytes = kWarps * kStages * kSlotBytes + kWarps * kStages * 8 + (kMaxSmemSeqs + 1) * 4 + 64;
 
 struct DecodeArgs {
     const __nv_bfloat16 *q;
@@ -143,47 +144,89 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
 
 // ------------------------------------------------------------------ split
 
-struct WarpRing {
-    uint8_t *slots;   // kStages * kSlotBytes
-    uint64_t *full;   // kStages barriers
+constexpr float kLn2 = 0.69314718055994530942f;
+
+// One unit of work: tokens [tok0, tok1) of sequence s, head h (split p).
+// Everything is warp-uniform except tbl0/tbl1/qv: lane l holds the physical
+// ids of the item's blocks l and 32 + l, and 16 bytes (8 dims) of the q row.
+struct Item {
+    int s, h, p, tok0, tok1, nt;  // nt: 16-token tiles (0: no item)
+    int tbl0, tbl1;
+    uint4 qv;
 };
 
-// Physical id of the block holding logical token `tok` of sequence s, or -1
-// (with the error bit set) when the table entry is out of range.
-__device__ __forceinline__ int resolve_block(const DecodeArgs &a, int s, int tok) {
-    const int lb = tok / a.block_size;
-    const int phys = __ldg(a.block_table + (size_t)s * a.max_blocks + lb);
-    return (phys >= 0 && phys < a.num_blocks) ? phys : -1;
-}
-
-__device__ __forceinline__ size_t tile_offset(const DecodeArgs &a, int phys, int h, int tok) {
-    // element offset of token `tok` of head h inside physical block phys
-    return (((size_t)phys * a.H + h) * a.block_size + (tok % a.block_size)) * kD;
-}
-
-// Lane 0: start the copy of tile `t` (tokens tok0 + 16 t ..) into slot.
-__device__ __forceinline__ void issue_tile(const DecodeArgs &a, const WarpRing &r, int slot, int s, int h,
-                                           int tok) {
-    const int phys = resolve_block(a, s, tok);
-    uint64_t *bar = r.full + slot;
-    if (phys < 0) {
-        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
-        mbar_arrive(bar);  // complete the phase without touching memory
+// Take the next item from the work counter (all lanes; lane 0 does the
+// atomic).  Loads the item's block-table entries and q row into registers
+// now, so neither is a dependent load later.
+__device__ __forceinline__ void fetch_item(const DecodeArgs &a, const int32_t *starts, int total, int lane,
+                                           int &s_hint, Item &it) {
+    int idx = 0;
+    if (lane == 0) idx = atomicAdd(a.counter, 1);
+    idx = __shfl_sync(0xffffffffu, idx, 0);
+    if (idx >= total) {
+        it.nt = 0;
         return;
     }
-    const size_t off = tile_offset(a, phys, h, tok);
-    uint8_t *dst = r.slots + slot * kSlotBytes;
+    const int k = idx / a.H;
+    it.h = idx - k * a.H;
+    // sequence holding split k: starts[s] <= k < starts[s + 1]
+    int lo = 0, hi = a.num_seqs - 1;
+    if (starts[s_hint] <= k && k < starts[s_hint + 1]) {
+        lo = s_hint;
+    } else {
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (starts[mid] <= k) lo = mid; else hi = mid - 1;
+        }
+    }
+    s_hint = it.s = lo;
+    it.p = k - starts[lo];
+    it.tok0 = it.p * a.split_tokens;
+    // independent loads: the length, the split's block ids (up to 64, read
+    // within the table row whatever the length), the q row
+    const int L = a.seq_lens[lo];
+    const int lb0 = it.tok0 / a.block_size;
+    const int room = a.max_blocks - lb0;
+    const int32_t *row = a.block_table + (size_t)lo * a.max_blocks + lb0;
+    const int t0 = lane < room ? __ldg(row + lane) : -1;
+    const int t1 = lane + 32 < room ? __ldg(row + 32 + lane) : -1;
+    it.qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)lo * a.H + it.h) * kD + 8 * (lane & 15));
+    it.tok1 = min(L, it.tok0 + a.split_tokens);
+    it.nt = (it.tok1 - it.tok0 + kTileTok - 1) / kTileTok;
+    const int nblk = (it.tok1 - it.tok0 + a.block_size - 1) / a.block_size;  // <= 64 by the split choice
+    it.tbl0 = lane < nblk ? t0 : -1;
+    it.tbl1 = lane + 32 < nblk ? t1 : -1;
+}
+
+// Physical block of tile t of the item (all lanes; -1 when out of range).
+__device__ __forceinline__ int tile_block(const DecodeArgs &a, const Item &it, int t) {
+    const int bi = (t * kTileTok) / a.block_size;  // tok0 is a multiple of block_size
+    const int v = __shfl_sync(0xffffffffu, bi < 32 ? it.tbl0 : it.tbl1, bi & 31);
+    return (v >= 0 && v < a.num_blocks) ? v : -1;
+}
+
+// Lane 0: start the copies of tile t of `it` into `slot` (or, for a block
+// outside the pool, complete the slot's phase without touching memory).
+__device__ __forceinline__ void issue_tile(const DecodeArgs &a, uint8_t *slots, uint64_t *full, int slot,
+                                           const Item &it, int t, int phys) {
+    uint64_t *bar = full + slot;
+    if (phys < 0) {
+        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+        mbar_arrive(bar);
+        return;
+    }
+    const int tok = it.tok0 + t * kTileTok;
+    const size_t off = (((size_t)phys * a.H + it.h) * a.block_size + (tok % a.block_size)) * kD;
+    uint8_t *dst = slots + slot * kSlotBytes;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(bar, kSlotBytes);
     bulk_g2s(dst, a.k_cache + off, kTileBytes, bar);
     bulk_g2s(dst + kTileBytes, a.v_cache + off, kTileBytes, bar);
 }
 
-constexpr float kLn2 = 0.69314718055994530942f;
-
 // Final bf16 row of O (o * inv_l, or zeros when o is null) and its LSE.
 // Lanes of half 0 hold dims 8*li .. 8*li+7.
-__device__ __forceinline__ void inv_l_store(const DecodeArgs &a, size_t sh, int li, int half, int lane,
+__device__ __forceinline__ void final_store(const DecodeArgs &a, size_t sh, int li, int half, int lane,
                                             const float *o, float inv_l, float lse) {
     if (half == 0) {
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -198,88 +241,153 @@ __device__ __forceinline__ void inv_l_store(const DecodeArgs &a, size_t sh, int 
     if (lane == 0) a.LSE[sh] = lse;
 }
 
+// Output of a finished item: the final row for a one-split sequence, else a
+// partial; the warp completing the last split of (s, h) merges in split order.
+__device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it, int lane, float m, float l,
+                                            float (&o)[8], bool saw_bad) {
+    const int half = lane >> 4, li = lane & 15;
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] += __shfl_xor_sync(0xffffffffu, o[c], 16);
+    const int nsplit = a.item_start[it.s + 1] - a.item_start[it.s];  // (L2-resident, once per item)
+    const size_t sh = (size_t)it.s * a.H + it.h;
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    if (nsplit == 1) {
+        if (saw_bad)
+            final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
+        else
+            final_store(a, sh, li, half, lane, o, inv_l, l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY);
+        return;
+    }
+    const size_t pidx = sh * a.max_splits + it.p;
+    if (half == 0) {
+        float4 *dst = reinterpret_cast<float4 *>(a.part_o + pidx * kD + 8 * li);
+        dst[0] = make_float4(o[0] * inv_l, o[1] * inv_l, o[2] * inv_l, o[3] * inv_l);
+        dst[1] = make_float4(o[4] * inv_l, o[5] * inv_l, o[6] * inv_l, o[7] * inv_l);
+    }
+    if (lane == 0) {
+        a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
+        if (saw_bad) atomicOr(a.seq_bad + it.s, 1);
+    }
+    __threadfence();  // partials (and the bad mark) before the completion count
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = (atomicAdd(a.done_cnt + sh, 1) == nsplit - 1);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence();
+    if (__ldcg(a.seq_bad + it.s)) {
+        final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
+        return;
+    }
+    const float *plse = a.part_lse + sh * a.max_splits;
+    float M = -INFINITY;
+    for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(plse + q));
+    float tot = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < nsplit; ++q) {
+        const float w = ex2_approx(__ldcg(plse + q) - M);
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sh * a.max_splits + q) * kD) + lane);
+        tot += w;
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+    }
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = packed;
+    if (lane == 0) a.LSE[sh] = tot > 0.f ? (M + __log2f(tot)) * kLn2 : -INFINITY;
+}
+
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    WarpRing ring;
-    ring.slots = smem + (size_t)wid * kStages * kSlotBytes;
-    ring.full = reinterpret_cast<uint64_t *>(smem + kWarps * kStages * kSlotBytes) + wid * kStages;
+    uint8_t *slots = smem + (size_t)wid * kStages * kSlotBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kWarps * kStages * kSlotBytes) + wid * kStages;
     if (lane == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(ring.full + i, 1);
+        for (int i = 0; i < kStages; ++i) mbar_init(full + i, 1);
         fence_barrier_init();
     }
     __syncwarp();
-
     const int half = lane >> 4, li = lane & 15;
     pdl_wait();  // the plan kernel's writes are visible from here on
-    const int total = a.item_start[a.num_seqs] * a.H;
-    uint32_t gtile = 0;  // tiles consumed by this warp so far (ring phase)
-    uint32_t pending = 0;  // lane 0: slots with a copy in flight
-    bool dead = false;
+    // per-sequence split offsets, staged in shared memory when they fit
+    const int32_t *starts = a.item_start;
+    if (a.num_seqs <= kMaxSmemSeqs) {
+        int32_t *st = reinterpret_cast<int32_t *>(smem + kWarps * kStages * kSlotBytes + kWarps * kStages * 8);
+        for (int i = threadIdx.x; i <= a.num_seqs; i += blockDim.x) st[i] = a.item_start[i];
+        __syncthreads();
+        starts = st;
+    }
+    const int total = starts[a.num_seqs] * a.H;
     int s_hint = 0;
 
-    while (!dead) {
-        int item = 0;
-        if (lane == 0) item = atomicAdd(a.counter, 1);
-        item = __shfl_sync(0xffffffffu, item, 0);
-        if (item >= total) break;
-        const int k = item / a.H, h = item - k * a.H;
-        // sequence holding split k: item_start[s] <= k < item_start[s + 1]
-        int lo = 0, hi = a.num_seqs - 1;
-        if (a.item_start[s_hint] <= k && k < a.item_start[s_hint + 1]) {
-            lo = hi = s_hint;
-        } else {
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (a.item_start[mid] <= k) lo = mid; else hi = mid - 1;
-            }
-        }
-        const int s = lo;
-        s_hint = s;
-        const int p = k - a.item_start[s];
-        const int L = a.seq_lens[s];
-        const int tok0 = p * a.split_tokens;
-        const int tok1 = min(L, tok0 + a.split_tokens);
-        const int nt = (tok1 - tok0 + kTileTok - 1) / kTileTok;
+    // The warp is a stream of 16-token tiles over consecutive items: the
+    // producer (lane 0's copies) runs kStages tiles ahead of the consumer,
+    // crossing into the next item (cur -> nxt) so the ring never drains.
+    Item cur, nxt;
+    fetch_item(a, starts, total, lane, s_hint, cur);
+    bool have_nxt = false, exhausted = (cur.nt == 0);
+    int pq = 0, pt = 0;           // producer: item (0 cur, 1 nxt) and next tile
+    uint32_t gi = 0, gc = 0;      // tiles issued / consumed by this warp
+    bool dead = false;
 
-        // q row for (s, h), 8 dims per lane, pre-scaled into log2 units
+    auto produce = [&]() -> bool {
+        for (;;) {
+            const int pnt = pq ? nxt.nt : cur.nt;
+            if (pt < pnt) {
+                const int phys = pq ? tile_block(a, nxt, pt) : tile_block(a, cur, pt);
+                if (lane == 0) issue_tile(a, slots, full, gi % kStages, pq ? nxt : cur, pt, phys);
+                ++pt;
+                ++gi;
+                return true;
+            }
+            if (pq == 1 || exhausted) return false;
+            fetch_item(a, starts, total, lane, s_hint, nxt);
+            if (nxt.nt == 0) {
+                exhausted = true;
+                return false;
+            }
+            have_nxt = true;
+            pq = 1;
+            pt = 0;
+        }
+    };
+
+    if (!exhausted) {
+        while (gi - gc < (uint32_t)kStages && produce()) {
+        }
+    }
+    while (!exhausted || cur.nt > 0) {
+        if (cur.nt == 0) break;
         float qf[8];
         {
-            const uint4 qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)s * a.H + h) * kD + 8 * li);
-            const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+            const uint32_t w[4] = {cur.qv.x, cur.qv.y, cur.qv.z, cur.qv.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 qf[2 * c] = bf16lo(w[c]) * a.scale_log2;
                 qf[2 * c + 1] = bf16hi(w[c]) * a.scale_log2;
             }
         }
-
-        // prologue: fill the ring
-        if (lane == 0) {
-            for (int t = 0; t < nt && t < kStages; ++t) {
-                const int slot = (gtile + t) % kStages;
-                issue_tile(a, ring, slot, s, h, tok0 + t * kTileTok);
-                pending |= 1u << slot;
-            }
-        }
-        __syncwarp();
-
         float m = -INFINITY, l = 0.f;
         float o[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) o[c] = 0.f;
         bool saw_bad = false;
-
-        for (int t = 0; t < nt; ++t, ++gtile) {
-            const int slot = gtile % kStages;
-            const uint32_t parity = (gtile / kStages) & 1u;
-            if (!mbar_wait(ring.full + slot, parity, a.err)) { dead = true; break; }
-            if (lane == 0) pending &= ~(1u << slot);
-            const int tok = tok0 + t * kTileTok;
-            const bool tile_ok = resolve_block(a, s, tok) >= 0;
+        for (int t = 0; t < cur.nt; ++t) {
+            const int slot = gc % kStages;
+            if (!mbar_wait(full + slot, (gc / kStages) & 1u, a.err)) {
+                dead = true;
+                break;
+            }
+            const int tok = cur.tok0 + t * kTileTok;
+            const bool tile_ok = tile_block(a, cur, t) >= 0;
             saw_bad |= !tile_ok;
             if (tile_ok) {
-                const uint8_t *kt = ring.slots + slot * kSlotBytes;
+                const uint8_t *kt = slots + slot * kSlotBytes;
                 const uint8_t *vt = kt + kTileBytes;
                 float sc[8];
 #pragma unroll
@@ -297,7 +405,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
                     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    sc[i] = (tok + r < tok1) ? acc : -INFINITY;
+                    sc[i] = (tok + r < cur.tok1) ? acc : -INFINITY;
                 }
                 float mt = sc[0];
 #pragma unroll
@@ -317,7 +425,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 2 * i + half;
-                    if (tok + r < tok1) {
+                    if (tok + r < cur.tok1) {
                         const uint4 vv = *reinterpret_cast<const uint4 *>(vt + r * (kD * 2) + li * 16);
                         const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
@@ -329,85 +437,24 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 }
                 m = m_new;
             }
-            __syncwarp();
-            if (lane == 0 && t + kStages < nt) {
-                issue_tile(a, ring, slot, s, h, tok + kStages * kTileTok);
-                pending |= 1u << slot;
-            }
-            __syncwarp();
+            ++gc;
+            __syncwarp();  // every lane is done with the slot before it is refilled
+            if (gi - gc < (uint32_t)kStages) produce();
         }
         if (dead) break;
-
-        // combine the two half-warps (same running max m)
-        l += __shfl_xor_sync(0xffffffffu, l, 16);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) o[c] += __shfl_xor_sync(0xffffffffu, o[c], 16);
-        const int nsplit = a.item_start[s + 1] - a.item_start[s];
-        const size_t sh = (size_t)s * a.H + h;
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        if (nsplit == 1) {
-            // whole sequence in this item: final result, no partial round trip
-            if (saw_bad) {
-                inv_l_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
-            } else {
-                inv_l_store(a, sh, li, half, lane, o, inv_l, l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY);
-            }
-            continue;
+        finish_item(a, cur, lane, m, l, o, saw_bad);
+        if (!have_nxt) break;
+        cur = nxt;
+        have_nxt = false;
+        pq = 0;
+        while (gi - gc < (uint32_t)kStages && produce()) {
         }
-        const size_t pidx = sh * a.max_splits + p;
-        if (half == 0) {
-            float4 *dst = reinterpret_cast<float4 *>(a.part_o + pidx * kD + 8 * li);
-            dst[0] = make_float4(o[0] * inv_l, o[1] * inv_l, o[2] * inv_l, o[3] * inv_l);
-            dst[1] = make_float4(o[4] * inv_l, o[5] * inv_l, o[6] * inv_l, o[7] * inv_l);
-        }
-        if (lane == 0) {
-            a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
-            if (saw_bad) atomicOr(a.seq_bad + s, 1);
-        }
-        __threadfence();  // partials (and the bad mark) before the completion count
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(a.done_cnt + sh, 1) == nsplit - 1);
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
-        // this warp finished the last split of (s, h): merge in split order
-        __threadfence();
-        if (__ldcg(a.seq_bad + s)) {
-            inv_l_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
-            continue;
-        }
-        const float *plse = a.part_lse + sh * a.max_splits;
-        float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(plse + q));
-        float tot = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < nsplit; ++q) {
-            const float w = ex2_approx(__ldcg(plse + q) - M);
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sh * a.max_splits + q) * kD) + lane);
-            tot += w;
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
-        const float inv = tot > 0.f ? 1.f / tot : 0.f;
-        uint2 packed;
-        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = packed;
-        if (lane == 0) a.LSE[sh] = tot > 0.f ? (M + __log2f(tot)) * kLn2 : -INFINITY;
     }
 
     // after a timeout: wait (bounded) for this warp's copies still in flight
     // so no bulk copy lands in shared memory after the CTA has exited
-    if (lane == 0 && pending) {
-        for (int i = 0; i < kStages; ++i) {
-            if (pending & (1u << i)) {
-                // the outstanding phase of slot i is the one after the last consumed
-                const uint32_t uses = gtile / kStages + ((uint32_t)i < gtile % kStages ? 1u : 0u);
-                mbar_wait(ring.full + i, uses & 1u, nullptr);
-            }
-        }
+    if (dead && lane == 0) {
+        for (uint32_t g = gc; g < gi; ++g) mbar_wait(full + g % kStages, (g / kStages) & 1u, nullptr);
     }
 }
 
@@ -436,7 +483,9 @@ int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_si
     const long long max_len = (long long)max_blocks * block_size;
     const long long work = (long long)num_seqs * H * max_len;
     long long split = 256;
-    while (split < max_len && work / split > 65536) split <<= 1;
+    // larger splits for large problems (bounded workspace), at most 64 blocks
+    // per split (the kernel keeps a split's block ids in two registers per lane)
+    while (split < max_len && work / split > 65536 && split * 2 <= 64LL * block_size) split <<= 1;
     return (int)split;
 }
 

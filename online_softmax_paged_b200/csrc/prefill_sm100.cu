@@ -60,8 +60,8 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = NQ * kTileBytes;
     static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-    // barriers: q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], done
-    static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], done
+    static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 };
@@ -203,6 +203,28 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint
     }
 }
 
+// Work unit u (a 256-row query block of one (b, h)) -> its block index and
+// (b, h); causal units are numbered longest first.
+__device__ __forceinline__ void unit_coords(const PrefillArgs &a, bool causal, int u, int &blk, int &bh) {
+    blk = causal ? (a.nblk - 1 - u / a.BH) : (u / a.BH);
+    bh = u % a.BH;
+}
+
+// The r-th unit of CTA c in snake order over rows of gridDim.x units
+// (row-major rows, every other row reversed), or -1 past the end.
+__device__ __forceinline__ int snake_unit(int r, int c, int G, int n_units) {
+    const int u = r * G + ((r & 1) ? (G - 1 - c) : c);
+    return u < n_units ? u : -1;
+}
+
+// Key tiles each query tile of unit (blk) visits; 0 when the tile is past N.
+__device__ __forceinline__ void tile_counts(const PrefillArgs &a, bool causal, int blk, int &n0, int &n1) {
+    const int n_kv_all = (a.N + BN - 1) / BN;
+    const int q0 = NQ * blk, q1 = NQ * blk + 1;
+    n0 = (q0 * BM >= a.N) ? 0 : (causal ? min(q0 + 1, n_kv_all) : n_kv_all);
+    n1 = (q1 * BM >= a.N) ? 0 : (causal ? min(q1 + 1, n_kv_all) : n_kv_all);
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -212,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *q_full = bars;
-    uint64_t *kv_full = bars + 2;
+    uint64_t *q_empty = q_full + 2;
+    uint64_t *kv_full = q_empty + 2;
     uint64_t *kv_empty = kv_full + C::kStages;
     uint64_t *s_full = kv_empty + C::kStages;
     uint64_t *p_full = s_full + 2;
@@ -222,31 +245,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMiscOff + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // work unit: longest causal query blocks first
-    const int lin = blockIdx.x;
-    const int blk = CAUSAL ? (a.nblk - 1 - lin / a.BH) : (lin / a.BH);
-    const int bh = lin % a.BH;
-    const int n_kv_all = (a.N + BN - 1) / BN;
-    int nkv[NQ];
-#pragma unroll
-    for (int i = 0; i < NQ; ++i) {
-        const int qt = NQ * blk + i;
-        nkv[i] = (qt * BM >= a.N) ? 0 : (CAUSAL ? min(qt + 1, n_kv_all) : n_kv_all);
-    }
-    const int nkv_max = max(nkv[0], nkv[1]);
+    const int G = gridDim.x, c = blockIdx.x;
+    const int n_units = a.nblk * a.BH;
 
     if (threadIdx.x == 0) {
-        mbar_init(&q_full[0], 1);
-        mbar_init(&q_full[1], 1);
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-        }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
             mbar_init(&o_full[i], 1);
+        }
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -269,32 +281,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             bool ok = true;
-            for (int i = 0; i < NQ; ++i) {
-                if (nkv[i] == 0) continue;
-                uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
-                mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
-                for (int b = 0; b < C::kBoxes; ++b)
-                    tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, (NQ * blk + i) * BM, bh);
-            }
-            const int n_loads = 2 * nkv_max;
-            int u = 0;
-            for (; u < n_loads && ok; ++u) {
-                const int slot = u % C::kStages;
-                if (u >= C::kStages) ok = wait_or_abort(&kv_empty[slot], ((u / C::kStages) - 1) & 1, a.err, abort_flag);
-                if (!ok) break;
-                const int j = u >> 1;
-                const CUtensorMap *tm = (u & 1) ? &tmV : &tmK;
-                uint8_t *dst = smem + C::kRingOff + slot * C::kTileBytes;
-                mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
-                for (int b = 0; b < C::kBoxes; ++b)
-                    tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, j * BN, bh);
+            uint32_t ukv = 0;         // K/V tiles loaded so far (ring position)
+            uint32_t qc[2] = {0, 0};  // Q tiles loaded so far, per query tile
+            for (int r = 0; ok; ++r) {
+                const int u = snake_unit(r, c, G, n_units);
+                if (u < 0) break;
+                int blk, bh, n0, n1;
+                unit_coords(a, CAUSAL, u, blk, bh);
+                tile_counts(a, CAUSAL, blk, n0, n1);
+                for (int i = 0; i < NQ && ok; ++i) {
+                    if ((i ? n1 : n0) == 0) continue;
+                    // the previous unit's QK^T products of this tile are done
+                    if (qc[i] > 0) ok = wait_or_abort(&q_empty[i], (qc[i] - 1) & 1, a.err, abort_flag);
+                    if (!ok) break;
+                    uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
+                    mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
+                    for (int b = 0; b < C::kBoxes; ++b)
+                        tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, (NQ * blk + i) * BM, bh);
+                    ++qc[i];
+                }
+                const int n_loads = 2 * max(n0, n1);
+                for (int v = 0; v < n_loads && ok; ++v, ++ukv) {
+                    const int slot = ukv % C::kStages;
+                    if (ukv >= (uint32_t)C::kStages)
+                        ok = wait_or_abort(&kv_empty[slot], ((ukv / C::kStages) - 1) & 1, a.err, abort_flag);
+                    if (!ok) break;
+                    const CUtensorMap *tm = (v & 1) ? &tmV : &tmK;
+                    uint8_t *dst = smem + C::kRingOff + slot * C::kTileBytes;
+                    mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+                    for (int b = 0; b < C::kBoxes; ++b)
+                        tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN, bh);
+                }
             }
             // copies still in flight must land before the CTA can exit: wait
-            // (bounded) for the newest phase of every slot that was loaded
-            for (int v = max(0, u - C::kStages); v < u; ++v)
+            // (bounded) for the newest phase of every slot and Q buffer loaded
+            const uint32_t first = ukv > (uint32_t)C::kStages ? ukv - C::kStages : 0u;
+            for (uint32_t v = first; v < ukv; ++v)
                 mbar_wait(&kv_full[v % C::kStages], (v / C::kStages) & 1, nullptr);
             for (int i = 0; i < NQ; ++i)
-                if (nkv[i] > 0) mbar_wait(&q_full[i], 0, nullptr);
+                if (qc[i] > 0) mbar_wait(&q_full[i], (qc[i] - 1) & 1, nullptr);
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
@@ -304,11 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_addr = smem_base + C::kQOff;
             const uint32_t ring_addr = smem_base + C::kRingOff;
             bool ok = true;
-            auto slot_addr = [&](int u) { return ring_addr + (u % C::kStages) * C::kTileBytes; };
-            auto wait_kv = [&](int u) {
+            uint32_t ukv = 0;             // K/V ring position (same order as the producer)
+            uint32_t qc[2] = {0, 0};      // Q tiles consumed, per query tile
+            uint32_t it[2] = {0, 0};      // key-tile iterations done, per query tile
+            auto slot_addr = [&](uint32_t u) { return ring_addr + (u % C::kStages) * C::kTileBytes; };
+            auto wait_kv = [&](uint32_t u) {
                 return wait_or_abort(&kv_full[u % C::kStages], (u / C::kStages) & 1, a.err, abort_flag);
             };
-            auto issue_s = [&](int i, int u) {
+            auto issue_s = [&](int i, uint32_t u) {
                 const uint32_t qa = q_addr + i * C::kTileBytes, ka = slot_addr(u);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
@@ -318,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&s_full[i]);
             };
-            auto issue_pv = [&](int i, int u, int j) {
+            auto issue_pv = [&](int i, uint32_t u, int j) {
                 const uint32_t va = slot_addr(u);
 #pragma unroll
                 for (int ks = 0; ks < BN / 16; ++ks) {
@@ -327,45 +355,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&o_full[i]);
             };
-            for (int i = 0; i < NQ && ok; ++i)
-                if (nkv[i] > 0) ok = wait_or_abort(&q_full[i], 0, a.err, abort_flag);
-            if (ok) ok = wait_kv(0);
-            if (ok) {
-                tc_fence_after();
-                for (int i = 0; i < NQ; ++i)
-                    if (nkv[i] > 0) issue_s(i, 0);
-                mma_commit(&kv_empty[0]);
-            }
-            for (int j = 0; j < nkv_max && ok; ++j) {
-                const int uV = 2 * j + 1, uK = 2 * j + 2;
-                ok = wait_kv(uV);
+            for (int r = 0; ok; ++r) {
+                const int u = snake_unit(r, c, G, n_units);
+                if (u < 0) break;
+                int blk, bh, n0, n1;
+                unit_coords(a, CAUSAL, u, blk, bh);
+                tile_counts(a, CAUSAL, blk, n0, n1);
+                const int nkv_max = max(n0, n1);
+                for (int i = 0; i < NQ && ok; ++i)
+                    if ((i ? n1 : n0) > 0) ok = wait_or_abort(&q_full[i], qc[i] & 1, a.err, abort_flag);
+                if (ok) ok = wait_kv(ukv);
                 if (!ok) break;
-                bool k_ready = false;
-                for (int i = 0; i < NQ && ok; ++i) {
-                    if (j >= nkv[i]) continue;
-                    ok = wait_or_abort(&p_full[i], j & 1, a.err, abort_flag);
+                tc_fence_after();
+                if (n0 > 0) issue_s(0, ukv);
+                if (n1 > 0) issue_s(1, ukv);
+                mma_commit(&kv_empty[ukv % C::kStages]);
+                for (int j = 0; j < nkv_max && ok; ++j) {
+                    const uint32_t uV = ukv + 2 * j + 1, uK = ukv + 2 * j + 2;
+                    ok = wait_kv(uV);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(i, uV, j);
-                    if (j + 1 < nkv[i]) {
+                    bool k_ready = false;
+                    for (int i = 0; i < NQ && ok; ++i) {
+                        const int ni = i ? n1 : n0;
+                        if (j >= ni) continue;
+                        ok = wait_or_abort(&p_full[i], (it[i] + j) & 1, a.err, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(i, uV, j);
+                        if (j + 1 < ni) {
+                            if (!k_ready) {
+                                ok = wait_kv(uK);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_s(i, uK);
+                        } else {
+                            // last QK^T of this tile was issued: Q_i may be reloaded
+                            mma_commit(&q_empty[i]);
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(&kv_empty[uV % C::kStages]);
+                    if (j + 1 < nkv_max) {
                         if (!k_ready) {
                             ok = wait_kv(uK);
                             if (!ok) break;
-                            tc_fence_after();
-                            k_ready = true;
                         }
-                        issue_s(i, uK);
+                        mma_commit(&kv_empty[uK % C::kStages]);
                     }
                 }
-                if (!ok) break;
-                mma_commit(&kv_empty[uV % C::kStages]);
-                if (j + 1 < nkv_max) {
-                    if (!k_ready) {
-                        ok = wait_kv(uK);
-                        if (!ok) break;
-                    }
-                    mma_commit(&kv_empty[uK % C::kStages]);
-                }
+                ukv += 2 * nkv_max;
+                it[0] += n0;
+                it[1] += n1;
+                if (n0 > 0) ++qc[0];
+                if (n1 > 0) ++qc[1];
             }
             // every MMA issued by this thread has completed before TMEM is freed
             mma_commit(done_bar);
@@ -375,109 +419,118 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ softmax
         const int i = warp >> 2;                 // query tile of this warpgroup
         const int quarter = warp & 3;            // TMEM lane quarter
-        const int r = quarter * 32 + lane;       // row inside the tile
-        const int qt = NQ * blk + i;
-        const int row = qt * BM + r;             // query row in the sequence
+        const int r_in = quarter * 32 + lane;    // row inside the tile
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_tm = tmem + lane_off + i * BN;
         const uint32_t o_tm = tmem + lane_off + 2 * BN + i * 128;
-        float m = -INFINITY, l = 0.f;
         bool ok = true;
-        const int my_nkv = i ? nkv[1] : nkv[0];
-        for (int j = 0; j < my_nkv; ++j) {
-            ok = wait_or_abort(&s_full[i], j & 1, a.err, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + 32 * c, sr[c]);
-            tmem_wait_ld();
-            // visible keys: col <= lim; only the causal diagonal tile and the
-            // sequence's last tile need masking
-            const bool masked = (CAUSAL && j == qt) || ((j + 1) * BN > a.N);
-            if (masked) {
-                int lim = BN - 1;
-                if (CAUSAL && j == qt) lim = r;
-                lim = min(lim, a.N - 1 - j * BN);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
-            }
-            float mxa[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mxa[k] = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                    const int k = (e >> 3) + 4 * (c & 1);
-                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
-                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
-                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 4]), __uint_as_float(sr[c][e + 5]));
-                    mxa[k] = max3(mxa[k], __uint_as_float(sr[c][e + 6]), __uint_as_float(sr[c][e + 7]));
-                }
-            const float mx = max3(max3(mxa[0], mxa[1], mxa[2]), max3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
-            const float mx2 = mx * a.scale_log2;
-            float m_ref = m;
-            if (mx2 > m + kRescaleThreshold) m_ref = mx2;
-            if (m_ref == -INFINITY) m_ref = 0.f;  // row with nothing visible yet
-            const float alpha = ex2_approx(m - m_ref);
-            const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
-            const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
-            uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-            if (masked)
-                exp_pack_store<false>(sr, s_tm, scale2, negm2, acc2);
-            else
-                exp_pack_store<true>(sr, s_tm, scale2, negm2, acc2);
-            float psum;
-            {
-                const uint64_t t2 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
-                float u0, u1;
-                f2_unpack(t2, u0, u1);
-                psum = u0 + u1;
-            }
-            l = l * alpha + psum;
-            const bool need = (m_ref != m) && j > 0;
-            if (__any_sync(0xffffffffu, need)) {
-                // PV(j-1) has completed: S(j) was issued after it and has landed
-                ok = wait_or_abort(&o_full[i], (j - 1) & 1, a.err, abort_flag);
+        uint32_t itc = 0;  // key-tile iterations done by this query tile so far
+        for (int rr = 0; ok; ++rr) {
+            const int u = snake_unit(rr, c, G, n_units);
+            if (u < 0) break;
+            int blk, bh, n0, n1;
+            unit_coords(a, CAUSAL, u, blk, bh);
+            tile_counts(a, CAUSAL, blk, n0, n1);
+            const int my_nkv = i ? n1 : n0;
+            const int qt = NQ * blk + i;
+            const int row = qt * BM + r_in;      // query row in the sequence
+            float m = -INFINITY, l = 0.f;
+            for (int j = 0; j < my_nkv; ++j) {
+                ok = wait_or_abort(&s_full[i], (itc + j) & 1, a.err, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
+                uint32_t sr[4][32];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t orr[32];
-                    tmem_ld32(o_tm + 32 * c, orr);
-                    tmem_wait_ld();
+                for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_tm + 32 * cc, sr[cc]);
+                tmem_wait_ld();
+                // visible keys: col <= lim; only the causal diagonal tile and the
+                // sequence's last tile need masking
+                const bool masked = (CAUSAL && j == qt) || ((j + 1) * BN > a.N);
+                if (masked) {
+                    int lim = BN - 1;
+                    if (CAUSAL && j == qt) lim = r_in;
+                    lim = min(lim, a.N - 1 - j * BN);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32(o_tm + 32 * c, orr);
+                    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * cc + e > lim) sr[cc][e] = __float_as_uint(-INFINITY);
                 }
+                float mxa[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mxa[k] = -INFINITY;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        const int k = (e >> 3) + 4 * (cc & 1);
+                        mxa[k] = max3(mxa[k], __uint_as_float(sr[cc][e]), __uint_as_float(sr[cc][e + 1]));
+                        mxa[k] = max3(mxa[k], __uint_as_float(sr[cc][e + 2]), __uint_as_float(sr[cc][e + 3]));
+                        mxa[k] = max3(mxa[k], __uint_as_float(sr[cc][e + 4]), __uint_as_float(sr[cc][e + 5]));
+                        mxa[k] = max3(mxa[k], __uint_as_float(sr[cc][e + 6]), __uint_as_float(sr[cc][e + 7]));
+                    }
+                const float mx =
+                    max3(max3(mxa[0], mxa[1], mxa[2]), max3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
+                const float mx2 = mx * a.scale_log2;
+                float m_ref = m;
+                if (mx2 > m + kRescaleThreshold) m_ref = mx2;
+                if (m_ref == -INFINITY) m_ref = 0.f;  // row with nothing visible yet
+                const float alpha = ex2_approx(m - m_ref);
+                const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
+                const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+                uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+                if (masked)
+                    exp_pack_store<false>(sr, s_tm, scale2, negm2, acc2);
+                else
+                    exp_pack_store<true>(sr, s_tm, scale2, negm2, acc2);
+                float psum;
+                {
+                    const uint64_t t2 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+                    float u0, u1;
+                    f2_unpack(t2, u0, u1);
+                    psum = u0 + u1;
+                }
+                l = l * alpha + psum;
+                const bool need = (m_ref != m) && j > 0;
+                if (__any_sync(0xffffffffu, need)) {
+                    // PV(j-1) has completed: S(j) was issued after it and has landed
+                    ok = wait_or_abort(&o_full[i], (itc + j - 1) & 1, a.err, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_tm + 32 * cc, orr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32(o_tm + 32 * cc, orr);
+                    }
+                }
+                m = m_ref;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[i]);
             }
-            m = m_ref;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[i]);
-        }
-        if (ok && my_nkv > 0) {
-            ok = wait_or_abort(&o_full[i], (my_nkv - 1) & 1, a.err, abort_flag);
-            if (ok) {
+            if (!ok) break;
+            if (my_nkv > 0) {
+                ok = wait_or_abort(&o_full[i], (itc + my_nkv - 1) & 1, a.err, abort_flag);
+                if (!ok) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 const bool live = row < a.N;
                 __nv_bfloat16 *orow = a.O + ((size_t)bh * a.N + (live ? row : 0)) * D;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t orr[32];
-                    tmem_ld32(o_tm + 32 * c, orr);
+                    tmem_ld32(o_tm + 32 * cc, orr);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
                     if (live) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cc);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
                             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
@@ -485,7 +538,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (live)
                     a.LSE[(size_t)bh * a.N + row] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+                // the O reads are complete before the next unit's first PV may
+                // overwrite O (ordered through p_full of that unit)
+                tc_fence_before();
             }
+            itc += my_nkv;
         }
         tc_fence_before();
     }
@@ -553,8 +610,15 @@ attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
     a.BH = BH;
     a.nblk = (p.N + NQ * BM - 1) / (NQ * BM);
     a.scale_log2 = p.scale * 1.4426950408889634f;
-    const long long grid = (long long)a.nblk * BH;
-    prefill_bf16_kernel<D, CAUSAL><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+    static int sm_count[64] = {0};
+    if (sm_count[dev] == 0 &&
+        cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ECUDA;
+    // persistent: one CTA per SM (the shared-memory footprint allows no more),
+    // each walking its units in snake order
+    const long long units = (long long)a.nblk * BH;
+    const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
+    prefill_bf16_kernel<D, CAUSAL><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
