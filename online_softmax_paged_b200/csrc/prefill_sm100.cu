@@ -178,16 +178,17 @@ constexpr int kPolyFrom = 5;  // 3 of every 8 pairs
 template <bool USE_POLY>
 __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint32_t s_tm, uint64_t scale2,
                                                uint64_t negm2, uint64_t (&acc2)[4]) {
+    // one 32-score chunk at a time: its 16 packed words are stored before the
+    // next chunk is exponentiated, so the chunk's registers are free again
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+    for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int c = 2 * h + (e >> 4), k = (e & 15) * 2;
+        for (int e = 0; e < 16; ++e) {
             const uint64_t x2 =
-                f2_fma(f2_pack(__uint_as_float(sr[c][k]), __uint_as_float(sr[c][k + 1])), scale2, negm2);
+                f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), scale2, negm2);
             uint64_t p2;
-            if (USE_POLY && (e & 7) >= kPolyFrom) {
+            if (USE_POLY && ((e + 16 * c) & 7) >= kPolyFrom) {
                 p2 = exp2_poly2(x2);
             } else {
                 float x0, x1;
@@ -199,7 +200,7 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint
             f2_unpack(p2, p0, p1);
             pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(s_tm + 32 * h, pk);
+        tmem_st16(s_tm + 16 * c, pk);
     }
 }
 
@@ -276,10 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA
-        if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
+        {
+            if (elect_one()) {
+                prefetch_tmap(&tmQ);
+                prefetch_tmap(&tmK);
+                prefetch_tmap(&tmV);
+            }
             bool ok = true;
             uint32_t ukv = 0;         // K/V tiles loaded so far (ring position)
             uint32_t qc[2] = {0, 0};  // Q tiles loaded so far, per query tile
@@ -295,9 +298,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (qc[i] > 0) ok = wait_or_abort(&q_empty[i], (qc[i] - 1) & 1, a.err, abort_flag);
                     if (!ok) break;
                     uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
-                    mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
-                    for (int b = 0; b < C::kBoxes; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, (NQ * blk + i) * BM, bh);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
+                        for (int b = 0; b < C::kBoxes; ++b)
+                            tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, (NQ * blk + i) * BM, bh);
+                    }
                     ++qc[i];
                 }
                 const int n_loads = 2 * max(n0, n1);
@@ -308,9 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     const CUtensorMap *tm = (v & 1) ? &tmV : &tmK;
                     uint8_t *dst = smem + C::kRingOff + slot * C::kTileBytes;
-                    mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
-                    for (int b = 0; b < C::kBoxes; ++b)
-                        tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN, bh);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+                        for (int b = 0; b < C::kBoxes; ++b)
+                            tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN, bh);
+                    }
                 }
             }
             // copies still in flight must land before the CTA can exit: wait
@@ -318,42 +325,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t first = ukv > (uint32_t)C::kStages ? ukv - C::kStages : 0u;
             for (uint32_t v = first; v < ukv; ++v)
                 mbar_wait(&kv_full[v % C::kStages], (v / C::kStages) & 1, nullptr);
-            for (int i = 0; i < NQ; ++i)
-                if (qc[i] > 0) mbar_wait(&q_full[i], (qc[i] - 1) & 1, nullptr);
+            if (qc[0] > 0) mbar_wait(&q_full[0], (qc[0] - 1) & 1, nullptr);
+            if (qc[1] > 0) mbar_wait(&q_full[1], (qc[1] - 1) & 1, nullptr);
+            __syncwarp();
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
+        {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
-            const uint32_t q_addr = smem_base + C::kQOff;
-            const uint32_t ring_addr = smem_base + C::kRingOff;
+            // base descriptors; per-slot and per-k-step offsets are added to the
+            // start-address field (16-byte units, no carry: smem < 256 KiB)
+            const uint64_t dq0 = desc_sw128(smem_base + C::kQOff, 16, 1024);
+            const uint64_t dq1 = desc_sw128(smem_base + C::kQOff + C::kTileBytes, 16, 1024);
+            const uint64_t dk = desc_sw128(smem_base + C::kRingOff, 16, 1024);
+            const uint64_t dv = desc_sw128(smem_base + C::kRingOff, kBoxBytes, 1024);
+            const uint32_t tm_s0 = tmem, tm_s1 = tmem + BN, tm_o0 = tmem + 2 * BN, tm_o1 = tmem + 2 * BN + 128;
             bool ok = true;
-            uint32_t ukv = 0;             // K/V ring position (same order as the producer)
-            uint32_t qc[2] = {0, 0};      // Q tiles consumed, per query tile
-            uint32_t it[2] = {0, 0};      // key-tile iterations done, per query tile
-            auto slot_addr = [&](uint32_t u) { return ring_addr + (u % C::kStages) * C::kTileBytes; };
+            uint32_t ukv = 0;              // K/V ring position (same order as the producer)
+            uint32_t qc0 = 0, qc1 = 0;     // Q tiles consumed, per query tile
+            uint32_t it0 = 0, it1 = 0;     // key-tile iterations done, per query tile
+            auto slot_off = [&](uint32_t u) -> uint64_t { return (uint64_t)(((u % C::kStages) * C::kTileBytes) >> 4); };
             auto wait_kv = [&](uint32_t u) {
                 return wait_or_abort(&kv_full[u % C::kStages], (u / C::kStages) & 1, a.err, abort_flag);
             };
             auto issue_s = [&](int i, uint32_t u) {
-                const uint32_t qa = q_addr + i * C::kTileBytes, ka = slot_addr(u);
+                const uint64_t da = i ? dq1 : dq0, db = dk + slot_off(u);
+                const uint32_t d_tm = i ? tm_s1 : tm_s0;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * kBoxBytes + (ks % 4) * 32;
-                    mma_ss(tmem + i * BN, desc_sw128(qa + off, 16, 1024), desc_sw128(ka + off, 16, 1024), idesc_qk,
-                           ks > 0);
+                if (elect_one()) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t off = (uint64_t)(((ks / 4) * kBoxBytes + (ks % 4) * 32) >> 4);
+                        mma_ss(d_tm, da + off, db + off, idesc_qk, ks > 0);
+                    }
+                    mma_commit(&s_full[i]);
                 }
-                mma_commit(&s_full[i]);
+                __syncwarp();
             };
             auto issue_pv = [&](int i, uint32_t u, int j) {
-                const uint32_t va = slot_addr(u);
+                const uint64_t db = dv + slot_off(u);
+                const uint32_t d_tm = i ? tm_o1 : tm_o0, p_tm = i ? tm_s1 : tm_s0;
+                if (elect_one()) {
 #pragma unroll
-                for (int ks = 0; ks < BN / 16; ++ks) {
-                    mma_ts(tmem + 2 * BN + i * 128, tmem + i * BN + ks * 8,
-                           desc_sw128(va + ks * 16 * 128, kBoxBytes, 1024), idesc_pv, (j > 0 || ks > 0));
+                    for (int ks = 0; ks < BN / 16; ++ks)
+                        mma_ts(d_tm, p_tm + ks * 8, db + (uint64_t)((ks * 16 * 128) >> 4), idesc_pv,
+                               (j > 0 || ks > 0));
+                    mma_commit(&o_full[i]);
                 }
-                mma_commit(&o_full[i]);
+                __syncwarp();
             };
             for (int r = 0; ok; ++r) {
                 const int u = snake_unit(r, c, G, n_units);
@@ -362,58 +382,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 unit_coords(a, CAUSAL, u, blk, bh);
                 tile_counts(a, CAUSAL, blk, n0, n1);
                 const int nkv_max = max(n0, n1);
-                for (int i = 0; i < NQ && ok; ++i)
-                    if ((i ? n1 : n0) > 0) ok = wait_or_abort(&q_full[i], qc[i] & 1, a.err, abort_flag);
+                if (n0 > 0) ok = wait_or_abort(&q_full[0], qc0 & 1, a.err, abort_flag);
+                if (ok && n1 > 0) ok = wait_or_abort(&q_full[1], qc1 & 1, a.err, abort_flag);
                 if (ok) ok = wait_kv(ukv);
                 if (!ok) break;
                 tc_fence_after();
                 if (n0 > 0) issue_s(0, ukv);
                 if (n1 > 0) issue_s(1, ukv);
-                mma_commit(&kv_empty[ukv % C::kStages]);
+                if (elect_one()) mma_commit(&kv_empty[ukv % C::kStages]);
                 for (int j = 0; j < nkv_max && ok; ++j) {
                     const uint32_t uV = ukv + 2 * j + 1, uK = ukv + 2 * j + 2;
                     ok = wait_kv(uV);
                     if (!ok) break;
                     bool k_ready = false;
-                    for (int i = 0; i < NQ && ok; ++i) {
+#pragma unroll
+                    for (int i = 0; i < NQ; ++i) {
                         const int ni = i ? n1 : n0;
-                        if (j >= ni) continue;
-                        ok = wait_or_abort(&p_full[i], (it[i] + j) & 1, a.err, abort_flag);
-                        if (!ok) break;
+                        if (!ok || j >= ni) continue;
+                        ok = wait_or_abort(&p_full[i], ((i ? it1 : it0) + j) & 1, a.err, abort_flag);
+                        if (!ok) continue;
                         tc_fence_after();
                         issue_pv(i, uV, j);
                         if (j + 1 < ni) {
                             if (!k_ready) {
                                 ok = wait_kv(uK);
-                                if (!ok) break;
+                                if (!ok) continue;
                                 tc_fence_after();
                                 k_ready = true;
                             }
                             issue_s(i, uK);
                         } else {
                             // last QK^T of this tile was issued: Q_i may be reloaded
-                            mma_commit(&q_empty[i]);
+                            if (elect_one()) mma_commit(&q_empty[i]);
                         }
                     }
                     if (!ok) break;
-                    mma_commit(&kv_empty[uV % C::kStages]);
+                    if (elect_one()) mma_commit(&kv_empty[uV % C::kStages]);
                     if (j + 1 < nkv_max) {
                         if (!k_ready) {
                             ok = wait_kv(uK);
                             if (!ok) break;
                         }
-                        mma_commit(&kv_empty[uK % C::kStages]);
+                        if (elect_one()) mma_commit(&kv_empty[uK % C::kStages]);
                     }
                 }
                 ukv += 2 * nkv_max;
-                it[0] += n0;
-                it[1] += n1;
-                if (n0 > 0) ++qc[0];
-                if (n1 > 0) ++qc[1];
+                it0 += n0;
+                it1 += n1;
+                if (n0 > 0) ++qc0;
+                if (n1 > 0) ++qc1;
             }
             // every MMA issued by this thread has completed before TMEM is freed
-            mma_commit(done_bar);
+            if (elect_one()) mma_commit(done_bar);
+            __syncwarp();
             mbar_wait(done_bar, 0, nullptr);
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ softmax
