@@ -47,7 +47,13 @@ namespace {
 constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // keys per tile
 constexpr int NQ = 2;          // query tiles per CTA
-constexpr int kThreads = 320;  // 2 softmax warpgroups + TMA warp + MMA warp
+constexpr int kThreads = 384;  // 2 softmax warpgroups + a producer warpgroup (TMA warp, MMA warp, 2 idle)
+// Register split (setmaxnreg, executed inside each role's branch): launched
+// at 168 per thread (384 x 168 = 64512); the producer warpgroup drops to 64
+// and each softmax warpgroup rises to 208: 128 x 64 + 256 x 208 = 61440.
+constexpr int kProducerRegs = 64;
+constexpr int kSoftmaxRegs = 208;
+static_assert(128 * kProducerRegs + 2 * 128 * kSoftmaxRegs <= kThreads * 168, "register split over budget");
 constexpr int kBoxCols = 64;   // bf16 elements per 128-byte swizzle row
 constexpr int kBoxBytes = 128 * 128;  // one box: 128 rows x 128 bytes
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -277,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
         {
             if (elect_one()) {
                 prefetch_tmap(&tmQ);
@@ -331,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
         {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
@@ -438,8 +446,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(done_bar, 0, nullptr);
             __syncwarp();
         }
+    } else if (warp >= 10) {
+        // idle warps of the producer warpgroup give their registers back
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
     } else {
         // ------------------------------------------------------------ softmax
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         const int i = warp >> 2;                 // query tile of this warpgroup
         const int quarter = warp & 3;            // TMEM lane quarter
         const int r_in = quarter * 32 + lane;    // row inside the tile

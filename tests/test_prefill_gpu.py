@@ -87,6 +87,25 @@ def test_bf16_large_scores_stay_exact():
     check_close(O, LSE, O_ref, L_ref, torch.bfloat16, "bf16 large scores")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_late_score_jump(causal):
+    """Keys from position 384 on score ~28 nats (~40 in log2 units) above the
+    first key tile: the reference max set by the first tile is too low by
+    more than 2^32, so the kernel must redo those tiles with their own max."""
+    inp = W.dense_inputs(1, 2, 900, 128, dtype=torch.bfloat16, seed=11, device="cuda", causal=causal)
+    Q, K = inp["Q"].clone(), inp["K"].clone()
+    Q[..., 0] = 2.0
+    K[..., 384:, 0] = 160.0
+    inp["Q"], inp["K"] = Q.contiguous(), K.contiguous()
+    O, LSE = _run(inp)
+    O_ref, L_ref = _full_oracle(inp)
+    # the jump is really there: rows past 384 see scores ~28 nats above the first tile's
+    assert L_ref[..., 500:].min() > 25.0
+    if causal:
+        assert L_ref[..., :384].max() < 15.0
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"late score jump causal={causal}")
+
+
 def test_prefill_2k_causal_full_size():
     """B=4 H=16 N=2048 d=128 causal bf16, seed 0: the launch the bench times.
     Four (b, h) heads against the oracle in full; every head for finiteness."""
