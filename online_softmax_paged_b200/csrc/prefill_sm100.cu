@@ -397,7 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 if (n0 > 0) issue_s(0, ukv);
                 if (n1 > 0) issue_s(1, ukv);
-                if (elect_one()) mma_commit(&kv_empty[ukv % C::kStages]);
+                if (elect_one()) {
+                    mma_commit(&kv_empty[ukv % C::kStages]);
+                    // a query tile with a single key tile has issued its only QK^T
+                    if (n0 == 1) mma_commit(&q_empty[0]);
+                    if (n1 == 1) mma_commit(&q_empty[1]);
+                }
                 for (int j = 0; j < nkv_max && ok; ++j) {
                     const uint32_t uV = ukv + 2 * j + 1, uK = ukv + 2 * j + 2;
                     ok = wait_kv(uV);
@@ -419,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 k_ready = true;
                             }
                             issue_s(i, uK);
-                        } else {
-                            // last QK^T of this tile was issued: Q_i may be reloaded
-                            if (elect_one()) mma_commit(&q_empty[i]);
+                            // that was the tile's last QK^T: Q_i may be reloaded once it
+                            // completes, so the next unit's Q load overlaps this unit
+                            if (j + 2 == ni && elect_one()) mma_commit(&q_empty[i]);
                         }
                     }
                     if (!ok) break;
