@@ -158,10 +158,16 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def kernel_sources_hash():
+KERNEL_SOURCES = {"prefill_bf16_kernel": ("prefill_sm100.cu", "ptx.cuh", "launch.h"),
+                  "decode_split_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h")}
+
+
+def kernel_sources_hash(kernel: str) -> str:
+    """Hash of the source files a kernel is built from (profiler counters are
+    only reported while these are unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "online_softmax_paged_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -176,7 +182,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{kernel}:{workload}")
-    if not e or e.get("sources") != kernel_sources_hash():
+    if not e or e.get("sources") != kernel_sources_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 

@@ -96,17 +96,20 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
         *a.counter = 0;
     }
     for (int i = tid; i < a.num_seqs * a.H; i += 1024) a.done_cnt[i] = 0;
-    for (int i = tid; i < a.num_seqs; i += 1024) a.seq_bad[i] = 0;
-    // sequences with no split: empty (L = 0) or an invalid length
-    for (int i = tid; i < a.num_seqs * a.H * (kD / 8); i += 1024) {
-        const int sh = i / (kD / 8), s = sh / a.H;
+    // sequences with no split (empty, or an invalid length): their rows are
+    // written here, one warp per such sequence
+    for (int s = wid; s < a.num_seqs; s += 32) {
         const int L = a.seq_lens[s];
         if (L > 0 && seq_len_ok(L, a)) continue;
-        const int c = i % (kD / 8);
-        reinterpret_cast<uint4 *>(a.O + (size_t)sh * kD)[c] = make_uint4(0u, 0u, 0u, 0u);
-        if (c == 0) a.LSE[sh] = -INFINITY;
-        if (c == 0 && (sh % a.H) == 0 && !seq_len_ok(L, a) && a.err) atomicOr(a.err, ATTN_DEVERR_SEQ_LEN);
+        if (lane == 0) {
+            a.seq_bad[s] = 0;
+            if (!seq_len_ok(L, a) && a.err) atomicOr(a.err, ATTN_DEVERR_SEQ_LEN);
+        }
+        for (int e = lane; e < a.H * (kD / 8); e += 32)
+            reinterpret_cast<uint4 *>(a.O + (size_t)s * a.H * kD)[e] = make_uint4(0u, 0u, 0u, 0u);
+        for (int h = lane; h < a.H; h += 32) a.LSE[(size_t)s * a.H + h] = -INFINITY;
     }
+    for (int i = tid; i < a.num_seqs; i += 1024) a.seq_bad[i] = 0;
     __syncthreads();
     for (int base = 0; base < a.num_seqs; base += 1024) {
         const int s = base + tid;
