@@ -9,6 +9,8 @@ A step is one call of the entry point on one batch of the workload:
   prefill_16k          attn_fwd, bf16 causal, B=1 H=32 N=16384 d=128 (x0.5)
   decode_uniform       paged_attn_decode, 64 seqs, H=32, bs=16, L~U[128,4096]
   decode_shared_prefix paged_attn_decode, 256 seqs, bs=32, 8-seq shared 512-token prefix
+  kv_append            paged_kv_append, 64 seqs x 512 new tokens (H=32, d=128, bs=16)
+  block_copy           paged_block_copy, 1024 block pairs (copy-on-write), 128 KiB per block
 The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
 decode_uniform, measured the same way in the same run, under "decode".
 
@@ -362,6 +364,145 @@ class Decode:
         return float(done_bytes), dt, f"{n} of {p.num_seqs} sequences of {self.name} (all heads)"
 
 
+class KVAppend:
+    """paged_kv_append of a prefill chunk: 64 sequences x 512 new tokens
+    (H=32, d=128, bs=16) written into fresh blocks drawn from a 20000-block
+    pool.  Work = bytes read + written (the copy-bandwidth convention)."""
+
+    def __init__(self, name, device, seed=0):
+        self.name = name
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        S, T, H, d, bs, pool = 64, 512, 32, 128, 16, 20000
+        self.k_cache = torch.zeros((pool, H, bs, d), dtype=torch.bfloat16, device=device)
+        self.v_cache = torch.zeros_like(self.k_cache)
+        mb = T // bs
+        self.table = torch.randperm(pool, generator=g, device=device)[:S * mb].view(S, mb).to(torch.int32).contiguous()
+        self.seq_ids = torch.arange(S, device=device, dtype=torch.int32).repeat_interleave(T).contiguous()
+        self.positions = torch.arange(T, device=device, dtype=torch.int32).repeat(S).contiguous()
+        self.k_new = torch.randn((S * T, H, d), generator=g, device=device).to(torch.bfloat16)
+        self.v_new = torch.randn((S * T, H, d), generator=g, device=device).to(torch.bfloat16)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.work = float(2 * 2 * self.k_new.numel() * 2)  # K and V, read and written
+        self.unit, self.scale_unit = "GB/s", 1e9
+        self.launches_per_step = 1
+        self.kernel = "kv_append_kernel"
+        self.cfg = dict(num_seqs=S, new_tokens_per_seq=T, H=H, d=d, block_size=bs, pool_blocks=pool)
+
+    def step(self, i, osp):
+        osp.paged_kv_append(self.k_new, self.v_new, self.seq_ids, self.positions, self.table, self.k_cache,
+                            self.v_cache, err_flag=self.err)
+
+    def config(self):
+        return {"workload": self.name, **self.cfg, "dtype": "bf16", "global_batch": self.cfg["num_seqs"],
+                "seq_len": self.cfg["new_tokens_per_seq"], "bytes_per_step": int(self.work),
+                "l2": "2.1 GiB of new K/V per step > L2"}
+
+    def e2e(self, osp, steps, device):
+        hk, hv = self.k_new.cpu().pin_memory(), self.v_new.cpu().pin_memory()
+        he = torch.zeros(1, dtype=torch.int32).pin_memory()
+        dk, dv = torch.empty_like(self.k_new), torch.empty_like(self.v_new)
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            osp.paged_kv_append(dk, dv, self.seq_ids, self.positions, self.table, self.k_cache, self.v_cache,
+                                err_flag=self.err)
+            he.copy_(self.err, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps, 2 * hk.numel() * 2, 4
+
+    def cpu_sample(self, budget_s):
+        import numpy as np
+        import oracle
+        S = self.cfg["num_seqs"]
+        T = self.cfg["new_tokens_per_seq"]
+        n = 4 * T  # four sequences' tokens
+        t0 = time.perf_counter()
+        kc = np.zeros((self.table[:4].numel() + 1, 32, 16, 128))
+        tbl = torch.arange(4 * (T // 16), dtype=torch.int32).view(4, T // 16).numpy()
+        oracle.kv_append(kc, kc, tbl, self.k_new[:n].float().cpu().numpy(), self.v_new[:n].float().cpu().numpy(),
+                         self.seq_ids[:n].cpu().numpy(), self.positions[:n].cpu().numpy(), 16)
+        dt = time.perf_counter() - t0
+        return self.work * n / (S * T), dt, f"4 of {S} sequences' tokens"
+
+
+class BlockCopy:
+    """paged_block_copy of 1024 (src, dst) pairs in a 20000-block pool
+    (H=32, d=128, bs=16: 128 KiB per block per cache).  Work = bytes read +
+    written."""
+
+    def __init__(self, name, device, seed=0):
+        self.name = name
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        pool, H, bs, d, n = 20000, 32, 16, 128, 1024
+        self.k_cache = torch.randn((pool, H, bs, d), generator=g, device=device).to(torch.bfloat16)
+        self.v_cache = torch.randn((pool, H, bs, d), generator=g, device=device).to(torch.bfloat16)
+        perm = torch.randperm(pool, generator=g, device=device).to(torch.int32)
+        self.src, self.dst = perm[:n].contiguous(), perm[n:2 * n].contiguous()
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.work = float(n * 2 * H * bs * d * 2 * 2)
+        self.unit, self.scale_unit = "GB/s", 1e9
+        self.launches_per_step = 1
+        self.kernel = "block_copy_kernel"
+        self.cfg = dict(pairs=n, H=H, d=d, block_size=bs, pool_blocks=pool)
+
+    def step(self, i, osp):
+        osp.paged_block_copy(self.k_cache, self.v_cache, self.src, self.dst, err_flag=self.err)
+
+    def config(self):
+        return {"workload": self.name, **self.cfg, "dtype": "bf16", "global_batch": self.cfg["pairs"],
+                "seq_len": self.cfg["block_size"], "bytes_per_step": int(self.work),
+                "l2": "268 MiB read per step > L2"}
+
+    def e2e(self, osp, steps, device):
+        hs, hd = self.src.cpu().pin_memory(), self.dst.cpu().pin_memory()
+        he = torch.zeros(1, dtype=torch.int32).pin_memory()
+        ds, dd = torch.empty_like(self.src), torch.empty_like(self.dst)
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            ds.copy_(hs, non_blocking=True)
+            dd.copy_(hd, non_blocking=True)
+            osp.paged_block_copy(self.k_cache, self.v_cache, ds, dd, err_flag=self.err)
+            he.copy_(self.err, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps, 2 * hs.numel() * 4, 4
+
+    def cpu_sample(self, budget_s):
+        import oracle
+        n = 16
+        kc = self.k_cache[:0]
+        src = self.src[:n].cpu().numpy()
+        dst = self.dst[:n].cpu().numpy()
+        idx = sorted(set(src.tolist()) | set(dst.tolist()))
+        remap = {b: i for i, b in enumerate(idx)}
+        sub_k = self.k_cache[idx].float().cpu().numpy()
+        sub_v = self.v_cache[idx].float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.block_copy(sub_k, sub_v, [remap[b] for b in src], [remap[b] for b in dst])
+        dt = time.perf_counter() - t0
+        return self.work * n / self.cfg["pairs"], dt, f"{n} of {self.cfg['pairs']} pairs"
+
+
 def make_workload(name, device, seed=0):
     if name == "prefill_2k":
         return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
@@ -369,6 +510,10 @@ def make_workload(name, device, seed=0):
         return Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
     if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small"):
         return Decode(name, device, seed)
+    if name == "kv_append":
+        return KVAppend(name, device, seed)
+    if name == "block_copy":
+        return BlockCopy(name, device, seed)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -590,7 +735,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_2k",
                     choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
-                             "decode_uniform_small"])
+                             "decode_uniform_small", "kv_append", "block_copy"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")

@@ -71,6 +71,7 @@ typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
 #define ATTN_DEVERR_BLOCK_TABLE 1 /* block_table entry outside [0, num_blocks) */
 #define ATTN_DEVERR_SEQ_LEN 2     /* seq_len < 0 or > max_blocks_per_seq * block_size */
 #define ATTN_DEVERR_TIMEOUT 4     /* a pipeline wait exceeded its iteration limit */
+#define ATTN_DEVERR_INDEX 8       /* a token's sequence id or position out of range */
 
 /*
  * Dense attention forward (prefill).
@@ -169,6 +170,50 @@ ATTN_API attn_status paged_attn_decode_noalloc(const void *q, const void *k_cach
                                       void *O, float *LSE,
                                       int num_seqs, int H, int d, int num_blocks, int max_blocks_per_seq,
                                       float scale, attn_dtype dt, int32_t *err_flag, attn_stream_t stream);
+
+/*
+ * Append new tokens' keys and values to the paged cache: the write that
+ * precedes decode ("一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解",
+ * section 三 核心原理: a new token goes into the sequence's current block,
+ * found through its block table; allocating that block is the caller's job).
+ *
+ * k_new, v_new : [num_tokens, H, d] of `dt`; token t belongs to sequence
+ *                seq_ids[t] at position positions[t] (int32 arrays).
+ * block_table  : int32 [num_seqs, max_blocks_per_seq], as for decode.
+ * k_cache,
+ * v_cache      : [num_blocks, H, block_size, d] of `dt`, written in place:
+ *                cache[block_table[s][pos / block_size], h, pos % block_size, :]
+ *                = new[t, h, :] for every head h.
+ * Supported    : ATTN_BF16 or ATTN_F32; d in {64, 128}; block_size in {16, 32}.
+ * Device checks: a sequence id or position out of range sets
+ *                ATTN_DEVERR_INDEX, a table entry outside [0, num_blocks)
+ *                sets ATTN_DEVERR_BLOCK_TABLE; that token is not written.
+ * Two tokens naming the same slot: which one lands is unspecified.
+ */
+ATTN_API attn_status paged_kv_append(const void *k_new, const void *v_new, const int32_t *seq_ids,
+                                     const int32_t *positions, int num_tokens, const int32_t *block_table,
+                                     int num_seqs, int max_blocks_per_seq, void *k_cache, void *v_cache,
+                                     int num_blocks, int H, int d, int block_size, attn_dtype dt,
+                                     int32_t *err_flag, attn_stream_t stream);
+
+/*
+ * Copy physical blocks for copy-on-write ("一文掌握大模型推理加速：
+ * FlashAttention与PagedAttention技术详解", section 三 内存共享机制: before a
+ * sequence writes into a block it shares, the block is copied to a new one
+ * and that sequence's table entry is redirected -- the table update and the
+ * reference counts are the caller's).
+ *
+ * For each pair i: block dst_blocks[i] of k_cache and of v_cache becomes a
+ * copy of block src_blocks[i] (all heads, all slots).  The destination
+ * blocks must be distinct and must not be sources of other pairs (the pairs
+ * run concurrently).  Caches [num_blocks, H, block_size, d] of `dt`.
+ * Supported    : ATTN_BF16 or ATTN_F32; d in {64, 128}; block_size in {16, 32}.
+ * Device checks: an id outside [0, num_blocks) sets ATTN_DEVERR_BLOCK_TABLE
+ *                and that pair is skipped.
+ */
+ATTN_API attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_t *src_blocks,
+                                      const int32_t *dst_blocks, int num_pairs, int num_blocks, int H, int d,
+                                      int block_size, attn_dtype dt, int32_t *err_flag, attn_stream_t stream);
 
 /*
  * Synchronise `stream`, read the device int32 at err_flag and return

@@ -16,7 +16,8 @@ import torch
 __all__ = [
     "AttnError", "attn_fwd", "paged_attn_decode", "paged_attn_decode_workspace_size",
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
-    "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "EXPORTED_SYMBOLS",
+    "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
+    "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -24,11 +25,12 @@ _LIB_PATH = os.path.join(_HERE, "libattn_sm100.so")
 
 ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_ECUDA, ATTN_EDEVICE = range(5)
 ATTN_F32, ATTN_BF16 = 0, 1
-ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT = 1, 2, 4
+ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_INDEX = 1, 2, 4, 8
 
 # every function include/attn.h declares
 EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
-                    "paged_attn_decode", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str")
+                    "paged_attn_decode", "paged_attn_decode_noalloc", "paged_kv_append", "paged_block_copy",
+                    "attn_read_error", "attn_status_str")
 
 # size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
 ATTN_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -68,6 +70,11 @@ def load():
     lib.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                               c_float, c_int, vp, vp]
     lib.paged_attn_decode_noalloc.restype = c_int
+    lib.paged_kv_append.argtypes = [vp, vp, vp, vp, c_int, vp, c_int, c_int, vp, vp, c_int, c_int, c_int, c_int,
+                                    c_int, vp, vp]
+    lib.paged_kv_append.restype = c_int
+    lib.paged_block_copy.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, vp, vp]
+    lib.paged_block_copy.restype = c_int
     lib.attn_read_error.argtypes = [vp, i32p, vp]
     lib.attn_read_error.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
@@ -204,6 +211,44 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, block_
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode_noalloc (scratch limit %d bytes)" % ATTN_NOALLOC_SCRATCH_BYTES)
     return O, LSE
+
+
+def paged_kv_append(k_new, v_new, seq_ids, positions, block_table, k_cache, v_cache, err_flag=None, stream=None):
+    """Write new tokens' K/V ([T, H, d]) into the paged caches in place.
+    seq_ids / positions: int32 [T]; block_table int32 [S, max_blocks_per_seq];
+    caches [num_blocks, H, block_size, d].  See include/attn.h."""
+    _check_cuda(k_new, v_new, seq_ids, positions, block_table, k_cache, v_cache, err_flag)
+    T, H, d = k_new.shape
+    if v_new.shape != k_new.shape or k_cache.shape != v_cache.shape or k_cache.shape[1] != H or \
+            k_cache.shape[3] != d or k_new.dtype != k_cache.dtype or v_new.dtype != k_cache.dtype:
+        raise ValueError("k_new/v_new [T, H, d] and caches [num_blocks, H, block_size, d] of one dtype")
+    if seq_ids.dtype != torch.int32 or positions.dtype != torch.int32 or block_table.dtype != torch.int32:
+        raise ValueError("seq_ids, positions and block_table must be int32")
+    for t in (k_new, v_new, seq_ids, positions, block_table, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    st = load().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(seq_ids), _ptr(positions), T, _ptr(block_table),
+                                block_table.shape[0], block_table.shape[1], _ptr(k_cache), _ptr(v_cache),
+                                k_cache.shape[0], H, d, k_cache.shape[2], _dtype_code(k_cache.dtype),
+                                _ptr(err_flag), _stream(stream, k_cache.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_kv_append")
+
+
+def paged_block_copy(k_cache, v_cache, src_blocks, dst_blocks, err_flag=None, stream=None):
+    """Copy physical blocks src -> dst in both caches (copy-on-write); the
+    destinations must be distinct and not sources.  See include/attn.h."""
+    _check_cuda(k_cache, v_cache, src_blocks, dst_blocks, err_flag)
+    if src_blocks.dtype != torch.int32 or dst_blocks.dtype != torch.int32 or src_blocks.shape != dst_blocks.shape:
+        raise ValueError("src_blocks and dst_blocks: int32 of one length")
+    if k_cache.shape != v_cache.shape or not (k_cache.is_contiguous() and v_cache.is_contiguous()):
+        raise ValueError("caches must be contiguous [num_blocks, H, block_size, d] of one shape")
+    nb, H, bs, d = k_cache.shape
+    st = load().paged_block_copy(_ptr(k_cache), _ptr(v_cache), _ptr(src_blocks.contiguous()),
+                                 _ptr(dst_blocks.contiguous()), src_blocks.numel(), nb, H, d, bs,
+                                 _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_block_copy")
 
 
 def attn_read_error(err_flag, stream=None) -> int:

@@ -70,6 +70,41 @@ attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_
     return osp::launch_paged_decode(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+attn_status paged_kv_append(const void *k_new, const void *v_new, const int32_t *seq_ids, const int32_t *positions,
+                            int num_tokens, const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                            void *k_cache, void *v_cache, int num_blocks, int H, int d, int block_size,
+                            attn_dtype dt, int32_t *err_flag, attn_stream_t stream) {
+    if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
+    if (num_tokens < 0 || num_seqs < 1 || max_blocks_per_seq < 1 || num_blocks < 1 || H < 1) return ATTN_EINVAL;
+    if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return ATTN_EUNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return ATTN_EINVAL;
+    if (num_tokens == 0) return ATTN_OK;
+    if (!k_new || !v_new || !seq_ids || !positions || !block_table || !k_cache || !v_cache) return ATTN_EINVAL;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return ATTN_EINVAL;
+    if (((uintptr_t)seq_ids & 3u) || ((uintptr_t)positions & 3u) || ((uintptr_t)block_table & 3u)) return ATTN_EINVAL;
+    osp::AppendLaunch p{k_new,      v_new, seq_ids, positions, block_table, k_cache, v_cache, num_tokens, num_seqs,
+                        max_blocks_per_seq, num_blocks, H, d, block_size, dt == ATTN_BF16 ? 2 : 4, err_flag};
+    return osp::launch_kv_append(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_t *src_blocks, const int32_t *dst_blocks,
+                             int num_pairs, int num_blocks, int H, int d, int block_size, attn_dtype dt,
+                             int32_t *err_flag, attn_stream_t stream) {
+    if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
+    if (num_pairs < 0 || num_blocks < 1 || H < 1) return ATTN_EINVAL;
+    if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return ATTN_EUNSUPPORTED;
+    if (num_pairs > 0x7fffffff / 2) return ATTN_EINVAL;
+    if (num_pairs == 0) return ATTN_OK;
+    if (!k_cache || !v_cache || !src_blocks || !dst_blocks) return ATTN_EINVAL;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return ATTN_EINVAL;
+    if (((uintptr_t)src_blocks & 3u) || ((uintptr_t)dst_blocks & 3u)) return ATTN_EINVAL;
+    osp::CopyLaunch p{k_cache, v_cache, src_blocks, dst_blocks, num_pairs, num_blocks, H, d, block_size,
+                      dt == ATTN_BF16 ? 2 : 4, err_flag};
+    return osp::launch_block_copy(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream) {
     if (!err_flag) return ATTN_EINVAL;
     int32_t v = 0;

@@ -1,0 +1,136 @@
+// kv_cache_ops.cu -- the two KV-cache writes around paged decode: appending
+// new tokens' keys/values into block-table-addressed slots, and the block copy
+// of copy-on-write.
+//
+// Method (pages): "一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解"
+// section 三 核心原理 -- a new token's K/V goes into its sequence's current
+// block (the block table maps the logical block to a physical one), and
+// sequences sharing a prompt point at the same physical blocks until one
+// writes, when the block is first copied (写时复制).  "第 2 章核心模块：
+// FlashAttention-2 与 PagedAttention 实现解析" section 2.2 (block table lookup).
+//
+// Both are pure data movement (HBM-bound): 16-byte vector loads and stores,
+// one CTA per token (append) or per (block, K|V) (copy).  Out-of-range ids are
+// skipped on the device and reported through err_flag, never dereferenced.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace osp {
+namespace {
+
+struct AppendArgs {
+    const uint8_t *k_new, *v_new;
+    const int32_t *seq_ids, *positions, *block_table;
+    uint8_t *k_cache, *v_cache;
+    int32_t *err;
+    int num_seqs, max_blocks, num_blocks, H, block_size;
+    int row_bytes;  // d * element size (a multiple of 16)
+};
+
+__global__ void __launch_bounds__(256) kv_append_kernel(AppendArgs a) {
+    __shared__ long long dst_row;  // element row index of (phys, h = 0, slot), or -1
+    const int t = blockIdx.x;
+    if (threadIdx.x == 0) {
+        const int s = a.seq_ids[t], pos = a.positions[t];
+        long long r = -1;
+        if (s < 0 || s >= a.num_seqs || pos < 0 || (long long)pos >= (long long)a.max_blocks * a.block_size) {
+            if (a.err) atomicOr(a.err, ATTN_DEVERR_INDEX);
+        } else {
+            const int phys = a.block_table[(size_t)s * a.max_blocks + pos / a.block_size];
+            if (phys < 0 || phys >= a.num_blocks) {
+                if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+            } else {
+                r = (long long)phys * a.H * a.block_size + pos % a.block_size;
+            }
+        }
+        dst_row = r;
+    }
+    __syncthreads();
+    const long long r0 = dst_row;
+    if (r0 < 0) return;
+    const int cpr = a.row_bytes / 16;  // 16-byte chunks per head row
+    const int per = a.H * cpr;
+    for (int c = threadIdx.x; c < 2 * per; c += blockDim.x) {
+        const int which = c >= per;
+        const int rem = c - which * per;
+        const int h = rem / cpr, q = rem - h * cpr;
+        const uint8_t *src = (which ? a.v_new : a.k_new) + ((size_t)t * a.H + h) * a.row_bytes + 16 * q;
+        uint8_t *dst = (which ? a.v_cache : a.k_cache) +
+                       ((size_t)r0 + (size_t)h * a.block_size) * a.row_bytes + 16 * q;
+        *reinterpret_cast<uint4 *>(dst) = __ldg(reinterpret_cast<const uint4 *>(src));
+    }
+}
+
+struct CopyArgs {
+    uint8_t *k_cache, *v_cache;
+    const int32_t *src, *dst;
+    int32_t *err;
+    int num_blocks;
+    long long block_bytes;  // H * block_size * d * element size (a multiple of 16)
+};
+
+// blockIdx.x: pair, blockIdx.y: 0 = K, 1 = V.  Each thread moves 4 x 16 bytes
+// per round so several loads are in flight before the first store.
+__global__ void __launch_bounds__(512) block_copy_kernel(CopyArgs a) {
+    const int i = blockIdx.x;
+    const int s = a.src[i], d = a.dst[i];
+    if (s < 0 || s >= a.num_blocks || d < 0 || d >= a.num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+        return;
+    }
+    uint8_t *base = blockIdx.y ? a.v_cache : a.k_cache;
+    const uint4 *from = reinterpret_cast<const uint4 *>(base + (size_t)s * a.block_bytes);
+    uint4 *to = reinterpret_cast<uint4 *>(base + (size_t)d * a.block_bytes);
+    const long long n = a.block_bytes / 16;
+    const int stride = blockDim.x;
+    long long k = threadIdx.x;
+    for (; k + 3 * stride < n; k += 4 * stride) {
+        const uint4 x0 = from[k], x1 = from[k + stride], x2 = from[k + 2 * stride], x3 = from[k + 3 * stride];
+        to[k] = x0;
+        to[k + stride] = x1;
+        to[k + 2 * stride] = x2;
+        to[k + 3 * stride] = x3;
+    }
+    for (; k < n; k += stride) to[k] = from[k];
+}
+
+}  // namespace
+
+attn_status launch_kv_append(const AppendLaunch &p, cudaStream_t stream) {
+    AppendArgs a;
+    a.k_new = static_cast<const uint8_t *>(p.k_new);
+    a.v_new = static_cast<const uint8_t *>(p.v_new);
+    a.seq_ids = p.seq_ids;
+    a.positions = p.positions;
+    a.block_table = p.block_table;
+    a.k_cache = static_cast<uint8_t *>(p.k_cache);
+    a.v_cache = static_cast<uint8_t *>(p.v_cache);
+    a.err = p.err_flag;
+    a.num_seqs = p.num_seqs;
+    a.max_blocks = p.max_blocks;
+    a.num_blocks = p.num_blocks;
+    a.H = p.H;
+    a.block_size = p.block_size;
+    a.row_bytes = p.d * p.elem_bytes;
+    kv_append_kernel<<<p.num_tokens, 256, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream) {
+    CopyArgs a;
+    a.k_cache = static_cast<uint8_t *>(p.k_cache);
+    a.v_cache = static_cast<uint8_t *>(p.v_cache);
+    a.src = p.src_blocks;
+    a.dst = p.dst_blocks;
+    a.err = p.err_flag;
+    a.num_blocks = p.num_blocks;
+    a.block_bytes = (long long)p.H * p.block_size * p.d * p.elem_bytes;
+    block_copy_kernel<<<dim3(p.num_pairs, 2), 512, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+}  // namespace osp

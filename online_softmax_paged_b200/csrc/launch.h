@@ -31,7 +31,24 @@ struct DecodeLaunch {
     int32_t *err_flag;
 };
 
+struct AppendLaunch {
+    const void *k_new, *v_new;
+    const int32_t *seq_ids, *positions, *block_table;
+    void *k_cache, *v_cache;
+    int num_tokens, num_seqs, max_blocks, num_blocks, H, d, block_size, elem_bytes;
+    int32_t *err_flag;
+};
+
+struct CopyLaunch {
+    void *k_cache, *v_cache;
+    const int32_t *src_blocks, *dst_blocks;
+    int num_pairs, num_blocks, H, d, block_size, elem_bytes;
+    int32_t *err_flag;
+};
+
 attn_status launch_dense_f32(const DenseLaunch &p, cudaStream_t stream);
+attn_status launch_kv_append(const AppendLaunch &p, cudaStream_t stream);
+attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream);
 attn_status launch_prefill_bf16(const DenseLaunch &p, cudaStream_t stream);
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream);
 

@@ -14,7 +14,9 @@ from .attention import (  # noqa: F401
     attention_flops,
     attention_head,
     attention_online_tiled,
+    block_copy,
     gather_paged,
+    kv_append,
     merge_partials,
     paged_decode,
     scores,

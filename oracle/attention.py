@@ -260,3 +260,53 @@ def attention_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
     diagonal, N(N+1)/2 pairs per head ([技术详解] §一: O(n^2 d) time)."""
     pairs = N * (N + 1) // 2 if causal else N * N
     return 4.0 * B * H * d * pairs
+
+
+def kv_append(k_cache, v_cache, block_table, k_new, v_new, seq_ids, positions, block_size: int):
+    """Write new tokens' keys/values into the paged cache (copy; float64 or any
+    dtype is kept).
+
+    [技术详解] §三 "核心原理" (a new token goes into the sequence's current
+    block, found through its block table) and [实现解析] §2.2 (logical block
+    -> physical block).  Token t of sequence seq_ids[t] at position
+    positions[t] lands in physical block block_table[s][pos // block_size],
+    slot pos % block_size, for every head.  Returns new arrays; a token whose
+    sequence, position or table entry is out of range is skipped and reported
+    in the returned list of skipped token indices.
+    """
+    k_out = np.array(k_cache, copy=True)
+    v_out = np.array(v_cache, copy=True)
+    num_blocks = k_out.shape[0]
+    S, mb = np.asarray(block_table).shape
+    skipped = []
+    for t in range(len(seq_ids)):
+        s, pos = int(seq_ids[t]), int(positions[t])
+        if not (0 <= s < S and 0 <= pos < mb * block_size):
+            skipped.append(t)
+            continue
+        phys = int(block_table[s][pos // block_size])
+        if not (0 <= phys < num_blocks):
+            skipped.append(t)
+            continue
+        k_out[phys, :, pos % block_size, :] = k_new[t]
+        v_out[phys, :, pos % block_size, :] = v_new[t]
+    return k_out, v_out, skipped
+
+
+def block_copy(k_cache, v_cache, src_blocks, dst_blocks):
+    """Copy-on-write step: physical block src -> dst (all heads, all slots) for
+    each pair, in pair order ([技术详解] §三 内存共享机制: a write to a shared
+    block first copies it to a new block).  Pairs with an id out of range are
+    skipped and reported."""
+    k_out = np.array(k_cache, copy=True)
+    v_out = np.array(v_cache, copy=True)
+    n = k_out.shape[0]
+    skipped = []
+    for i, (a, b) in enumerate(zip(src_blocks, dst_blocks)):
+        a, b = int(a), int(b)
+        if not (0 <= a < n and 0 <= b < n):
+            skipped.append(i)
+            continue
+        k_out[b] = k_cache[a]
+        v_out[b] = v_cache[a]
+    return k_out, v_out, skipped

@@ -367,3 +367,87 @@ def test_unmutated_copy_passes_pins():
     pin_golden_dense(attn)
     pin_torch_sdpa(attn)
     pin_closed_forms(attn)
+
+
+# --------------------------------------------------------------------------
+# KV-cache write and copy-on-write block copy
+# --------------------------------------------------------------------------
+
+def _pool(nb=10, H=2, bs=4, d=3, seed=60):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((nb, H, bs, d)), rng.standard_normal((nb, H, bs, d))
+
+
+def test_kv_append_python_loops():
+    """Token t goes to cache[table[s][pos // bs], h, pos % bs, :] for every
+    head, element by element."""
+    kc, vc = _pool()
+    table = np.array([[3, 7, -1], [0, 9, 2]])
+    rng = np.random.default_rng(61)
+    seq_ids = np.array([0, 1, 1, 0, 1])
+    pos = np.array([0, 5, 11, 6, 4])
+    kn = rng.standard_normal((5, 2, 3))
+    vn = rng.standard_normal((5, 2, 3))
+    k2, v2, skipped = oracle.kv_append(kc, vc, table, kn, vn, seq_ids, pos, 4)
+    assert skipped == []
+    kref, vref = kc.copy(), vc.copy()
+    for t in range(5):
+        blk = table[seq_ids[t]][pos[t] // 4]
+        for h in range(2):
+            for c in range(3):
+                kref[blk, h, pos[t] % 4, c] = kn[t, h, c]
+                vref[blk, h, pos[t] % 4, c] = vn[t, h, c]
+    np.testing.assert_array_equal(k2, kref)
+    np.testing.assert_array_equal(v2, vref)
+    assert (kc == _pool()[0]).all()  # input not modified
+
+
+def test_kv_append_then_gather_round_trip():
+    """Writing a sequence token by token then resolving the table by copy
+    gives back exactly the written rows (gather_paged is pinned above)."""
+    kc = np.zeros((8, 2, 4, 3))
+    vc = np.zeros((8, 2, 4, 3))
+    table = np.array([[5, 1, 6]])
+    L = 10
+    rng = np.random.default_rng(62)
+    kn = rng.standard_normal((L, 2, 3))
+    vn = rng.standard_normal((L, 2, 3))
+    order = rng.permutation(L)  # order of writes does not matter
+    k2, v2, _ = oracle.kv_append(kc, vc, table, kn[order], vn[order], np.zeros(L, int), order, 4)
+    np.testing.assert_array_equal(oracle.gather_paged(k2, table[0], L, 4), kn.transpose(1, 0, 2))
+    np.testing.assert_array_equal(oracle.gather_paged(v2, table[0], L, 4), vn.transpose(1, 0, 2))
+
+
+def test_kv_append_skips_out_of_range():
+    kc, vc = _pool()
+    table = np.array([[3, 11]])  # 11 is outside the 10-block pool
+    kn = np.ones((4, 2, 3))
+    k2, v2, skipped = oracle.kv_append(kc, vc, table, kn, kn, np.array([0, 0, 1, 0]), np.array([1, 5, 0, 8]), 4)
+    assert skipped == [1, 2, 3]  # bad table entry, bad sequence id, position past the table
+    assert (k2[3, :, 1] == 1).all()
+    k_check = kc.copy()
+    k_check[3, :, 1] = 1
+    np.testing.assert_array_equal(k2, k_check)
+
+
+def test_block_copy_and_copy_on_write():
+    kc, vc = _pool(seed=63)
+    k2, v2, skipped = oracle.block_copy(kc, vc, [4, 2, 12], [6, 8, 0])
+    assert skipped == [2]
+    np.testing.assert_array_equal(k2[6], kc[4])
+    np.testing.assert_array_equal(v2[8], vc[2])
+    others = [b for b in range(10) if b not in (6, 8)]
+    np.testing.assert_array_equal(k2[others], kc[others])
+    # copy-on-write: two sequences share physical block 4; sequence 1 writes
+    # into it, so the block is first copied to a free block 7 and its table
+    # entry redirected; sequence 0 still sees the old contents
+    table = np.array([[4, 1], [4, 3]])
+    k3, v3, _ = oracle.block_copy(kc, vc, [4], [7])
+    table[1, 0] = 7
+    newk = np.full((1, 2, 3), 9.0)
+    k4, v4, _ = oracle.kv_append(k3, v3, table, newk, newk, np.array([1]), np.array([2]), 4)
+    g0 = oracle.gather_paged(k4, table[0], 4, 4)
+    g1 = oracle.gather_paged(k4, table[1], 4, 4)
+    np.testing.assert_array_equal(g0, kc[4])
+    assert (g1[:, 2] == 9).all()
+    np.testing.assert_array_equal(np.delete(g1, 2, axis=1), np.delete(kc[4], 2, axis=1))
