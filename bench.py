@@ -9,6 +9,7 @@ A step is one call of the entry point on one batch of the workload:
   prefill_16k          attn_fwd, bf16 causal, B=1 H=32 N=16384 d=128 (x0.5)
   decode_uniform       paged_attn_decode, 64 seqs, H=32, bs=16, L~U[128,4096]
   decode_shared_prefix paged_attn_decode, 256 seqs, bs=32, 8-seq shared 512-token prefix
+  decode_gqa_g4/_g8    paged_attn_decode_gqa, decode_uniform with 32 query heads over 8 / 4 K/V heads
   kv_append            paged_kv_append, 64 seqs x 512 new tokens (H=32, d=128, bs=16)
   block_copy           paged_block_copy, 1024 block pairs (copy-on-write), 128 KiB per block
 The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
@@ -270,6 +271,16 @@ class Decode:
         self.name = name
         if name == "decode_uniform":
             self.p = W.paged_uniform(device=device, seed=seed, **W.DECODE_UNIFORM)
+        elif name in ("decode_gqa_g4", "decode_gqa_g8"):
+            # the uniform decode workload with 32 query heads over 8 (or 4)
+            # key/value heads: grouped-query attention
+            Hkv = 8 if name == "decode_gqa_g4" else 4
+            base = W.paged_uniform(device=device, seed=seed, **{**W.DECODE_UNIFORM, "H": Hkv})
+            g = torch.Generator(device=device)
+            g.manual_seed(seed + 1)
+            q = torch.randn((base.num_seqs, 32, base.d), generator=g, device=device).to(torch.bfloat16)
+            self.p = W.PagedInputs(q, base.k_cache, base.v_cache, base.block_table, base.seq_lens,
+                                   base.block_size, base.scale)
         elif name == "decode_uniform_small":
             # 16 sequences of the uniform workload in a 4000-block pool (1 GiB
             # of K/V, still above L2): the case profiler captures run on
@@ -277,8 +288,11 @@ class Decode:
                                                                    "pool": 4000})
         else:
             self.p = W.paged_shared_prefix(device=device, seed=seed, **W.DECODE_SHARED_PREFIX)
-        self.logical = W.logical_kv_bytes(self.p)
-        self.unique = W.unique_kv_bytes(self.p)
+        self.gqa = self.p.k_cache.shape[1] != self.p.q.shape[1]
+        kv = W.PagedInputs(self.p.q[:, :self.p.k_cache.shape[1]], self.p.k_cache, self.p.v_cache,
+                           self.p.block_table, self.p.seq_lens, self.p.block_size, self.p.scale)
+        self.logical = W.logical_kv_bytes(kv)   # K/V bytes of the key/value heads attended
+        self.unique = W.unique_kv_bytes(kv)
         self.work = float(self.unique if name == "decode_shared_prefix" else self.logical)  # bytes per step
         self.O = torch.empty_like(self.p.q)
         self.LSE = torch.empty(self.p.q.shape[:2], dtype=torch.float32, device=device)
@@ -293,12 +307,14 @@ class Decode:
 
     def step(self, i, osp):
         p = self.p
-        osp.paged_attn_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.block_size, O=self.O,
-                              LSE=self.LSE, scale=p.scale, workspace=self.ws)
+        fn = osp.paged_attn_decode_gqa if self.gqa else osp.paged_attn_decode
+        fn(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.block_size, O=self.O, LSE=self.LSE,
+           scale=p.scale, workspace=self.ws)
 
     def config(self):
         p = self.p
-        c = {"workload": self.name, "num_seqs": p.num_seqs, "H": p.H, "d": p.d, "block_size": p.block_size,
+        c = {"workload": self.name, "num_seqs": p.num_seqs, "H": p.H, "H_kv": int(p.k_cache.shape[1]), "d": p.d,
+             "block_size": p.block_size,
              "pool_blocks": p.num_blocks, "dtype": "bf16", "global_batch": p.num_seqs,
              "seq_len": int(p.seq_lens.max().item()), "kv_bytes_logical": self.logical,
              "kv_bytes_unique": self.unique,
@@ -319,8 +335,9 @@ class Decode:
             dq.copy_(hq, non_blocking=True)
             dt.copy_(ht, non_blocking=True)
             ds.copy_(hs, non_blocking=True)
-            osp.paged_attn_decode(dq, p.k_cache, p.v_cache, dt, ds, p.block_size, O=self.O, LSE=self.LSE,
-                                  scale=p.scale, workspace=self.ws)
+            fn = osp.paged_attn_decode_gqa if self.gqa else osp.paged_attn_decode
+            fn(dq, p.k_cache, p.v_cache, dt, ds, p.block_size, O=self.O, LSE=self.LSE, scale=p.scale,
+               workspace=self.ws)
             ho.copy_(self.O, non_blocking=True)
             hl.copy_(self.LSE, non_blocking=True)
 
@@ -508,7 +525,7 @@ def make_workload(name, device, seed=0):
         return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
     if name == "prefill_16k":
         return Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
-    if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small"):
+    if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small", "decode_gqa_g4", "decode_gqa_g8"):
         return Decode(name, device, seed)
     if name == "kv_append":
         return KVAppend(name, device, seed)
@@ -735,7 +752,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_2k",
                     choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
-                             "decode_uniform_small", "kv_append", "block_copy"])
+                             "decode_uniform_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")

@@ -141,6 +141,27 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
                               int32_t *err_flag, attn_stream_t stream);
 
 /*
+ * Grouped-query paged decode: H_q query heads share H_kv key/value heads,
+ * query head h reading key/value head h / (H_q / H_kv) (multi-query attention
+ * is H_kv = 1).  The pages describe multi-head attention only; this is the
+ * same decode with the group mapping.
+ *
+ * q, O         : [num_seqs, H_q, d] bf16;   LSE : [num_seqs, H_q] fp32.
+ * k_cache,
+ * v_cache      : [num_blocks, H_kv, block_size, d] bf16.
+ * workspace    : paged_attn_decode_workspace_size(num_seqs, H_q, d, ...) bytes.
+ * Supported    : H_q / H_kv in {1, 2, 4, 8}; otherwise as paged_attn_decode
+ *                (whose behaviour, checks and determinism apply unchanged;
+ *                paged_attn_decode is this call with H_kv = H_q).
+ */
+ATTN_API attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
+                                           const int32_t *block_table, const int32_t *seq_lens, int block_size,
+                                           void *O, float *LSE, int num_seqs, int H_q, int H_kv, int d,
+                                           int num_blocks, int max_blocks_per_seq, float scale, attn_dtype dt,
+                                           void *workspace, size_t workspace_bytes, int32_t *err_flag,
+                                           attn_stream_t stream);
+
+/*
  * Paged decode without a workspace argument, for callers that cannot
  * allocate device memory (code running where cudaMalloc is not permitted or
  * not wanted, e.g. inside an allocator or pool callback, in a process whose

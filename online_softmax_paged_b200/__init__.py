@@ -17,7 +17,7 @@ __all__ = [
     "AttnError", "attn_fwd", "paged_attn_decode", "paged_attn_decode_workspace_size",
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
-    "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy",
+    "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,8 @@ ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_I
 
 # every function include/attn.h declares
 EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
-                    "paged_attn_decode", "paged_attn_decode_noalloc", "paged_kv_append", "paged_block_copy",
+                    "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_kv_append",
+                    "paged_block_copy",
                     "attn_read_error", "attn_status_str")
 
 # size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
@@ -67,6 +68,9 @@ def load():
     lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                       c_float, c_int, vp, c_size, vp, vp]
     lib.paged_attn_decode.restype = c_int
+    lib.paged_attn_decode_gqa.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
+                                          c_int, c_float, c_int, vp, c_size, vp, vp]
+    lib.paged_attn_decode_gqa.restype = c_int
     lib.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                               c_float, c_int, vp, vp]
     lib.paged_attn_decode_noalloc.restype = c_int
@@ -175,6 +179,40 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=
                                   _ptr(err_flag), _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode")
+    return O, LSE
+
+
+def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size, O=None, LSE=None, scale=None,
+                          workspace=None, err_flag=None, stream=None):
+    """Grouped-query paged decode: q [S, H_q, d], caches [num_blocks, H_kv,
+    block_size, d] with H_q / H_kv in {1, 2, 4, 8}.  See include/attn.h."""
+    _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, workspace, err_flag)
+    S, Hq, d = q.shape
+    nb, Hkv, bs, dk = k_cache.shape
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if k_cache.shape != v_cache.shape or bs != block_size or dk != d:
+        raise ValueError("caches must be [num_blocks, H_kv, block_size, d]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mb = block_table.shape[1]
+    need = paged_attn_decode_workspace_size(S, Hq, d, mb, block_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load().paged_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                      int(block_size), _ptr(O), _ptr(LSE), S, Hq, Hkv, d, nb, mb, float(scale),
+                                      _dtype_code(q.dtype), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _ptr(err_flag),
+                                      _stream(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_attn_decode_gqa")
     return O, LSE
 
 

@@ -44,18 +44,23 @@ int paged_attn_decode_split_tokens(int num_seqs, int H, int d, int max_blocks_pe
     return osp::decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size);
 }
 
-attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
-                              const int32_t *seq_lens, int block_size, void *O, float *LSE, int num_seqs, int H,
-                              int d, int num_blocks, int max_blocks_per_seq, float scale, attn_dtype dt,
-                              void *workspace, size_t workspace_bytes, int32_t *err_flag, attn_stream_t stream) {
+namespace {
+
+attn_status decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                        const int32_t *seq_lens, int block_size, void *O, float *LSE, int num_seqs, int H, int Hkv,
+                        int d, int num_blocks, int max_blocks_per_seq, float scale, attn_dtype dt, void *workspace,
+                        size_t workspace_bytes, int32_t *err_flag, attn_stream_t stream) {
     if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
-    if (num_seqs < 0 || H < 1 || num_blocks < 1 || max_blocks_per_seq < 1) return ATTN_EINVAL;
+    if (num_seqs < 0 || H < 1 || Hkv < 1 || num_blocks < 1 || max_blocks_per_seq < 1) return ATTN_EINVAL;
+    if (H % Hkv) return ATTN_EINVAL;
+    const int G = H / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_EUNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
     if (dt != ATTN_BF16) return ATTN_EUNSUPPORTED;
     if (d != 128) return ATTN_EUNSUPPORTED;
     if (block_size != 16 && block_size != 32) return ATTN_EUNSUPPORTED;
     if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return ATTN_EINVAL;
-    if ((long long)num_blocks * H * block_size * d > (1LL << 46)) return ATTN_EINVAL;
+    if ((long long)num_blocks * Hkv * block_size * d > (1LL << 46)) return ATTN_EINVAL;
     if (num_seqs == 0) return ATTN_OK;
     if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !O || !LSE || !workspace) return ATTN_EINVAL;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(O) || !aligned16(workspace))
@@ -66,8 +71,27 @@ attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_
         return ATTN_EINVAL;
     osp::DecodeLaunch p{q,        k_cache,  v_cache, block_table, seq_lens,         O,          LSE,
                         num_seqs, H,        d,       num_blocks,  max_blocks_per_seq, block_size, scale,
-                        workspace, err_flag};
+                        workspace, err_flag, Hkv};
     return osp::launch_paged_decode(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                              const int32_t *seq_lens, int block_size, void *O, float *LSE, int num_seqs, int H,
+                              int d, int num_blocks, int max_blocks_per_seq, float scale, attn_dtype dt,
+                              void *workspace, size_t workspace_bytes, int32_t *err_flag, attn_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE, num_seqs, H, H, d,
+                       num_blocks, max_blocks_per_seq, scale, dt, workspace, workspace_bytes, err_flag, stream);
+}
+
+attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *block_table, const int32_t *seq_lens, int block_size, void *O,
+                                  float *LSE, int num_seqs, int H_q, int H_kv, int d, int num_blocks,
+                                  int max_blocks_per_seq, float scale, attn_dtype dt, void *workspace,
+                                  size_t workspace_bytes, int32_t *err_flag, attn_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE, num_seqs, H_q, H_kv, d,
+                       num_blocks, max_blocks_per_seq, scale, dt, workspace, workspace_bytes, err_flag, stream);
 }
 
 attn_status paged_kv_append(const void *k_new, const void *v_new, const int32_t *seq_ids, const int32_t *positions,

@@ -48,11 +48,19 @@ namespace {
 constexpr int kD = 128;                         // head dim supported here
 constexpr int kTileTok = 16;                    // tokens per pipeline tile
 constexpr int kTileBytes = kTileTok * kD * 2;   // 4 KiB of K (or of V)
-constexpr int kWarps = 12;                      // workers per CTA
 constexpr int kStages = 2;                      // ring slots per worker
 constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
 constexpr int kMaxSmemSeqs = 4096;  // split offsets staged in shared memory up to this many sequences
-constexpr int kSmemBytes = kWarps * kStages * kSlotBytes + kWarps * kStages * 8 + (kMaxSmemSeqs + 1) * 4 + 64;
+// Workers per CTA: 12 for one query head per key/value head, fewer for
+// larger groups (each worker holds G query rows, accumulators and maxima).
+template <int G>
+struct Warps {
+    static constexpr int value = G >= 4 ? 8 : 12;
+};
+template <int W>
+constexpr int smem_bytes() {
+    return W * kStages * kSlotBytes + W * kStages * 8 + (kMaxSmemSeqs + 1) * 4 + 64;
+}
 
 struct DecodeArgs {
     const __nv_bfloat16 *q;
@@ -71,6 +79,7 @@ struct DecodeArgs {
     float *part_lse;      // [num_seqs, H, max_splits] log2 units
     float *part_o;        // [num_seqs, H, max_splits, d] normalised
     int num_seqs, H, num_blocks, max_blocks, block_size, split_tokens, max_splits;
+    int Hkv;              // key/value heads; H (query heads) = Hkv * G
     float scale_log2;     // scale * log2(e)
 };
 
@@ -149,9 +158,11 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
 
 constexpr float kLn2 = 0.69314718055994530942f;
 
-// One unit of work: tokens [tok0, tok1) of sequence s, head h (split p).
-// Everything is warp-uniform except tbl0/tbl1/qv: lane l holds the physical
-// ids of the item's blocks l and 32 + l, and 16 bytes (8 dims) of the q row.
+// One unit of work: tokens [tok0, tok1) of sequence s, key/value head h
+// (split p); with a group of G query heads per key/value head it serves query
+// heads h*G .. h*G+G-1.  Everything is warp-uniform except tbl0/tbl1/qv: lane
+// l holds the physical ids of the item's blocks l and 32 + l, and (G == 1)
+// 16 bytes (8 dims) of the q row.
 struct Item {
     int s, h, p, tok0, tok1, nt;  // nt: 16-token tiles (0: no item)
     int tbl0, tbl1;
@@ -161,6 +172,7 @@ struct Item {
 // Take the next item from the work counter (all lanes; lane 0 does the
 // atomic).  Loads the item's block-table entries and q row into registers
 // now, so neither is a dependent load later.
+template <int G>
 __device__ __forceinline__ void fetch_item(const DecodeArgs &a, const int32_t *starts, int total, int lane,
                                            int &s_hint, Item &it) {
     int idx = 0;
@@ -170,8 +182,8 @@ __device__ __forceinline__ void fetch_item(const DecodeArgs &a, const int32_t *s
         it.nt = 0;
         return;
     }
-    const int k = idx / a.H;
-    it.h = idx - k * a.H;
+    const int k = idx / a.Hkv;
+    it.h = idx - k * a.Hkv;
     // sequence holding split k: starts[s] <= k < starts[s + 1]
     int lo = 0, hi = a.num_seqs - 1;
     if (starts[s_hint] <= k && k < starts[s_hint + 1]) {
@@ -193,7 +205,7 @@ __device__ __forceinline__ void fetch_item(const DecodeArgs &a, const int32_t *s
     const int32_t *row = a.block_table + (size_t)lo * a.max_blocks + lb0;
     const int t0 = lane < room ? __ldg(row + lane) : -1;
     const int t1 = lane + 32 < room ? __ldg(row + 32 + lane) : -1;
-    it.qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)lo * a.H + it.h) * kD + 8 * (lane & 15));
+    if (G == 1) it.qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)lo * a.H + it.h) * kD + 8 * (lane & 15));
     it.tok1 = min(L, it.tok0 + a.split_tokens);
     it.nt = (it.tok1 - it.tok0 + kTileTok - 1) / kTileTok;
     const int nblk = (it.tok1 - it.tok0 + a.block_size - 1) / a.block_size;  // <= 64 by the split choice
@@ -219,7 +231,7 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, uint8_t *slots, 
         return;
     }
     const int tok = it.tok0 + t * kTileTok;
-    const size_t off = (((size_t)phys * a.H + it.h) * a.block_size + (tok % a.block_size)) * kD;
+    const size_t off = (((size_t)phys * a.Hkv + it.h) * a.block_size + (tok % a.block_size)) * kD;
     uint8_t *dst = slots + slot * kSlotBytes;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(bar, kSlotBytes);
@@ -246,14 +258,14 @@ __device__ __forceinline__ void final_store(const DecodeArgs &a, size_t sh, int 
 
 // Output of a finished item: the final row for a one-split sequence, else a
 // partial; the warp completing the last split of (s, h) merges in split order.
-__device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it, int lane, float m, float l,
+__device__ __forceinline__ void finish_item(const DecodeArgs &a, int s, int hq, int p, int lane, float m, float l,
                                             float (&o)[8], bool saw_bad) {
     const int half = lane >> 4, li = lane & 15;
     l += __shfl_xor_sync(0xffffffffu, l, 16);
 #pragma unroll
     for (int c = 0; c < 8; ++c) o[c] += __shfl_xor_sync(0xffffffffu, o[c], 16);
-    const int nsplit = a.item_start[it.s + 1] - a.item_start[it.s];  // (L2-resident, once per item)
-    const size_t sh = (size_t)it.s * a.H + it.h;
+    const int nsplit = a.item_start[s + 1] - a.item_start[s];  // (L2-resident, once per item)
+    const size_t sh = (size_t)s * a.H + hq;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     if (nsplit == 1) {
         if (saw_bad)
@@ -262,7 +274,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it,
             final_store(a, sh, li, half, lane, o, inv_l, l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY);
         return;
     }
-    const size_t pidx = sh * a.max_splits + it.p;
+    const size_t pidx = sh * a.max_splits + p;
     if (half == 0) {
         float4 *dst = reinterpret_cast<float4 *>(a.part_o + pidx * kD + 8 * li);
         dst[0] = make_float4(o[0] * inv_l, o[1] * inv_l, o[2] * inv_l, o[3] * inv_l);
@@ -270,7 +282,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it,
     }
     if (lane == 0) {
         a.part_lse[pidx] = l > 0.f ? m + __log2f(l) : -INFINITY;
-        if (saw_bad) atomicOr(a.seq_bad + it.s, 1);
+        if (saw_bad) atomicOr(a.seq_bad + s, 1);
     }
     __threadfence();  // partials (and the bad mark) before the completion count
     __syncwarp();
@@ -279,7 +291,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it,
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
     __threadfence();
-    if (__ldcg(a.seq_bad + it.s)) {
+    if (__ldcg(a.seq_bad + s)) {
         final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
         return;
     }
@@ -305,7 +317,9 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, const Item &it,
     if (lane == 0) a.LSE[sh] = tot > 0.f ? (M + __log2f(tot)) * kLn2 : -INFINITY;
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
+template <int G>
+__global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(DecodeArgs a) {
+    constexpr int kWarps = Warps<G>::value;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     uint8_t *slots = smem + (size_t)wid * kStages * kSlotBytes;
@@ -325,14 +339,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         __syncthreads();
         starts = st;
     }
-    const int total = starts[a.num_seqs] * a.H;
+    const int total = starts[a.num_seqs] * a.Hkv;
     int s_hint = 0;
 
     // The warp is a stream of 16-token tiles over consecutive items: the
     // producer (lane 0's copies) runs kStages tiles ahead of the consumer,
     // crossing into the next item (cur -> nxt) so the ring never drains.
     Item cur, nxt;
-    fetch_item(a, starts, total, lane, s_hint, cur);
+    fetch_item<G>(a, starts, total, lane, s_hint, cur);
     bool have_nxt = false, exhausted = (cur.nt == 0);
     int pq = 0, pt = 0;           // producer: item (0 cur, 1 nxt) and next tile
     uint32_t gi = 0, gc = 0;      // tiles issued / consumed by this warp
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 return true;
             }
             if (pq == 1 || exhausted) return false;
-            fetch_item(a, starts, total, lane, s_hint, nxt);
+            fetch_item<G>(a, starts, total, lane, s_hint, nxt);
             if (nxt.nt == 0) {
                 exhausted = true;
                 return false;
@@ -366,19 +380,30 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     }
     while (!exhausted || cur.nt > 0) {
         if (cur.nt == 0) break;
-        float qf[8];
-        {
-            const uint32_t w[4] = {cur.qv.x, cur.qv.y, cur.qv.z, cur.qv.w};
+        // query rows of the group, 8 dims per lane, pre-scaled into log2 units
+        float qf[G][8];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            uint4 qv;
+            if (G == 1)
+                qv = cur.qv;
+            else
+                qv = *reinterpret_cast<const uint4 *>(a.q + ((size_t)cur.s * a.H + cur.h * G + g) * kD + 8 * li);
+            const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                qf[2 * c] = bf16lo(w[c]) * a.scale_log2;
-                qf[2 * c + 1] = bf16hi(w[c]) * a.scale_log2;
+                qf[g][2 * c] = bf16lo(w[c]) * a.scale_log2;
+                qf[g][2 * c + 1] = bf16hi(w[c]) * a.scale_log2;
             }
         }
-        float m = -INFINITY, l = 0.f;
-        float o[8];
+        float m[G], l[G], o[G][8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) o[c] = 0.f;
+        for (int g = 0; g < G; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) o[g][c] = 0.f;
+        }
         bool saw_bad = false;
         for (int t = 0; t < cur.nt; ++t) {
             const int slot = gc % kStages;
@@ -392,60 +417,77 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             if (tile_ok) {
                 const uint8_t *kt = slots + slot * kSlotBytes;
                 const uint8_t *vt = kt + kTileBytes;
-                float sc[8];
+                // scores of all G query heads: each K row is read and converted once
+                float sc[G][8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 2 * i + half;
                     const uint4 kv = *reinterpret_cast<const uint4 *>(kt + r * (kD * 2) + li * 16);
                     const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-                    float acc = 0.f;
+                    float kf[8];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        acc = fmaf(qf[2 * c], bf16lo(w[c]), acc);
-                        acc = fmaf(qf[2 * c + 1], bf16hi(w[c]), acc);
+                        kf[2 * c] = bf16lo(w[c]);
+                        kf[2 * c + 1] = bf16hi(w[c]);
                     }
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    sc[i] = (tok + r < cur.tok1) ? acc : -INFINITY;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc = fmaf(qf[g][c], kf[c], acc);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                        sc[g][i] = (tok + r < cur.tok1) ? acc : -INFINITY;
+                    }
                 }
-                float mt = sc[0];
 #pragma unroll
-                for (int i = 1; i < 8; ++i) mt = fmaxf(mt, sc[i]);
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                const float m_new = fmaxf(m, mt);
-                const float alpha = ex2_approx(m - m_new);
-                float psum = 0.f;
+                for (int g = 0; g < G; ++g) {
+                    float mt = sc[g][0];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    sc[i] = ex2_approx(sc[i] - m_new);
-                    psum += sc[i];
+                    for (int i = 1; i < 8; ++i) mt = fmaxf(mt, sc[g][i]);
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                    const float m_new = fmaxf(m[g], mt);
+                    const float alpha = ex2_approx(m[g] - m_new);
+                    float psum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        sc[g][i] = ex2_approx(sc[g][i] - m_new);
+                        psum += sc[g][i];
+                    }
+                    l[g] = l[g] * alpha + psum;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) o[g][c] *= alpha;
+                    m[g] = m_new;
                 }
-                l = l * alpha + psum;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) o[c] *= alpha;
+                // P V for all G heads: each V row is read and converted once
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 2 * i + half;
                     if (tok + r < cur.tok1) {
                         const uint4 vv = *reinterpret_cast<const uint4 *>(vt + r * (kD * 2) + li * 16);
                         const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+                        float vf[8];
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
-                            o[2 * c] = fmaf(sc[i], bf16lo(w[c]), o[2 * c]);
-                            o[2 * c + 1] = fmaf(sc[i], bf16hi(w[c]), o[2 * c + 1]);
+                            vf[2 * c] = bf16lo(w[c]);
+                            vf[2 * c + 1] = bf16hi(w[c]);
                         }
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) o[g][c] = fmaf(sc[g][i], vf[c], o[g][c]);
                     }
                 }
-                m = m_new;
             }
             ++gc;
             __syncwarp();  // every lane is done with the slot before it is refilled
             if (gi - gc < (uint32_t)kStages) produce();
         }
         if (dead) break;
-        finish_item(a, cur, lane, m, l, o, saw_bad);
+#pragma unroll
+        for (int g = 0; g < G; ++g) finish_item(a, cur.s, cur.h * G + g, cur.p, lane, m[g], l[g], o[g], saw_bad);
         if (!have_nxt) break;
         cur = nxt;
         have_nxt = false;
@@ -503,18 +545,40 @@ size_t decode_workspace_bytes(int num_seqs, int H, int d, int max_blocks, int bl
     return ws_layout(num_seqs, H, ms < 1 ? 1 : ms).total;
 }
 
+template <int G>
+attn_status launch_split(const DecodeArgs &a, int dev, int sms, cudaStream_t stream) {
+    constexpr int W = Warps<G>::value;
+    static bool attr_set[64] = {false};
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(decode_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem_bytes<W>()) != cudaSuccess)
+            return ATTN_ECUDA;
+        attr_set[dev] = true;
+    }
+    // the split kernel is a programmatic dependent of the plan: its launch and
+    // barrier set-up overlap the plan; griddepcontrol.wait orders the data
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(W * 32);
+    cfg.dynamicSmemBytes = smem_bytes<W>();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_split_kernel<G>, a) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     static int sm_count[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ECUDA;
     if (dev < 0 || dev >= 64) return ATTN_ECUDA;
-    if (sm_count[dev] == 0) {
-        if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return ATTN_ECUDA;
-        if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes) != cudaSuccess)
-            return ATTN_ECUDA;
-    }
+    if (sm_count[dev] == 0 &&
+        cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ECUDA;
+    const int G = p.H / p.Hkv;
     DecodeArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(p.q);
     a.k_cache = static_cast<const __nv_bfloat16 *>(p.k_cache);
@@ -526,6 +590,7 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.err = p.err_flag;
     a.num_seqs = p.num_seqs;
     a.H = p.H;
+    a.Hkv = p.Hkv;
     a.num_blocks = p.num_blocks;
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
@@ -544,20 +609,13 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
 
     decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-    // the split kernel is a programmatic dependent of the plan: its launch and
-    // barrier set-up overlap the plan; griddepcontrol.wait orders the data
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sm_count[dev]);
-    cfg.blockDim = dim3(kWarps * 32);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_split_kernel, a) != cudaSuccess) return ATTN_ECUDA;
-    return ATTN_OK;
+    switch (G) {
+        case 1: return launch_split<1>(a, dev, sm_count[dev], stream);
+        case 2: return launch_split<2>(a, dev, sm_count[dev], stream);
+        case 4: return launch_split<4>(a, dev, sm_count[dev], stream);
+        case 8: return launch_split<8>(a, dev, sm_count[dev], stream);
+    }
+    return ATTN_EUNSUPPORTED;
 }
 
 }  // namespace osp

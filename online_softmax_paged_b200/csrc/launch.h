@@ -29,6 +29,7 @@ struct DecodeLaunch {
     float scale;
     void *workspace;
     int32_t *err_flag;
+    int Hkv;  // key/value heads (H / Hkv in {1, 2, 4, 8})
 };
 
 struct AppendLaunch {

@@ -211,14 +211,20 @@ def gather_paged(cache, block_table_row, L: int, block_size: int) -> np.ndarray:
 def paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int, scale: float, seqs=None):
     """Paged decode oracle: one query token per sequence.
 
-    q [S, H, d]; caches [num_blocks, H, block_size, d]; block_table
+    q [S, Hq, d]; caches [num_blocks, Hkv, block_size, d] with Hq a multiple
+    of Hkv (query head h reads key/value head h // (Hq / Hkv): grouped-query
+    attention; Hq == Hkv is plain multi-head attention); block_table
     [S, max_blocks_per_seq]; seq_lens [S].  For each sequence the keys and
-    values are first copied into contiguous [H, L, d] arrays
+    values are first copied into contiguous [Hkv, L, d] arrays
     (:func:`gather_paged`), then the dense definition runs with one query row
     and no mask ([区别] Q2: paging changes storage, not the math; reading 4).
-    Returns O [S, H, d], LSE [S, H]; sequences not in ``seqs`` stay NaN.
+    Returns O [S, Hq, d], LSE [S, Hq]; sequences not in ``seqs`` stay NaN.
     """
     S, H, d = q.shape
+    Hkv = k_cache.shape[1]
+    if H % Hkv:
+        raise ValueError("query heads must be a multiple of key/value heads")
+    G = H // Hkv
     O = np.full((S, H, v_cache.shape[3]), np.nan)
     LSE = np.full((S, H), np.nan)
     for s in (range(S) if seqs is None else seqs):
@@ -226,7 +232,8 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, block_size: int, sc
         Ks = gather_paged(k_cache, block_table[s], L, block_size)
         Vs = gather_paged(v_cache, block_table[s], L, block_size)
         for h in range(H):
-            o, lse = attention_head(np.asarray(q[s, h:h + 1], dtype=np.float64), Ks[h], Vs[h], False, scale)
+            o, lse = attention_head(np.asarray(q[s, h:h + 1], dtype=np.float64), Ks[h // G], Vs[h // G], False,
+                                    scale)
             O[s, h] = o[0]
             LSE[s, h] = lse[0]
     return O, LSE

@@ -180,3 +180,47 @@ def test_decode_equals_dense_last_row():
     torch.cuda.synchronize()
     assert (O[0].float() - Od[0, :, L - 1].float()).abs().max().item() <= 2e-2
     assert (LSE[0] - Ld[0, :, L - 1]).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("G,bs", [(2, 16), (4, 32), (8, 16), (4, 16)])
+def test_gqa_decode_full(G, bs):
+    """Grouped-query decode: H_q = 32 query heads over 32 / G key/value heads,
+    lengths 0..3000 (edge lengths included), against the grouped oracle."""
+    osp = _osp()
+    Hkv = 32 // G
+    lens = [0, 1, 17, 255, 256, 257, 1000, 3000, 2048, 5]
+    p = W.paged_uniform(H=Hkv, d=128, block_size=bs, pool=1200, len_hi=3000, seed=12 + G, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(40 + G)
+    q = torch.randn((len(lens), 32, 128), generator=g, device="cuda").to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = osp.paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, bs, scale=p.scale,
+                                       err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    O_ref, L_ref = oracle.paged_decode(to64(q), DeviceCache(p.k_cache), DeviceCache(p.v_cache),
+                                       p.block_table.cpu().numpy(), p.seq_lens.cpu().numpy(), bs, p.scale)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"gqa G={G} bs={bs}")
+    # placement shuffle: bit-identical
+    p2 = W.shuffle_placement(p, seed=3)
+    O2, L2 = osp.paged_attn_decode_gqa(q, p2.k_cache, p2.v_cache, p2.block_table, p2.seq_lens, bs, scale=p.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
+
+
+def test_gqa_group_one_is_multi_head():
+    osp = _osp()
+    p = W.paged_uniform(num_seqs=9, H=8, d=128, block_size=16, pool=900, len_lo=1, len_hi=1500, seed=30,
+                        device="cuda")
+    O1, L1 = _decode(p)
+    O2, L2 = osp.paged_attn_decode_gqa(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, 16, scale=p.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+def test_gqa_decode_bad_group_rejected():
+    osp = _osp()
+    p = W.paged_uniform(num_seqs=2, H=4, d=128, block_size=16, pool=100, len_lo=1, len_hi=100, seed=31,
+                        device="cuda")
+    q = torch.zeros((2, 12, 128), dtype=torch.bfloat16, device="cuda")  # group of 3
+    with pytest.raises(osp.AttnError):
+        osp.paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, 16)

@@ -451,3 +451,20 @@ def test_block_copy_and_copy_on_write():
     np.testing.assert_array_equal(g0, kc[4])
     assert (g1[:, 2] == 9).all()
     np.testing.assert_array_equal(np.delete(g1, 2, axis=1), np.delete(kc[4], 2, axis=1))
+
+
+def test_paged_decode_grouped_query_heads():
+    """Grouped-query decode: query head h reads key/value head h // G.  Pinned
+    against the multi-head oracle on a cache whose heads are repeated G times
+    (each query head then has its own copy of its group's keys)."""
+    q, kc, vc, table, lens, bs = _tiny_paged(21, S=5, H=2, d=3)
+    G = 3
+    qg = np.random.default_rng(22).standard_normal((5, 2 * G, 3))
+    O, L = oracle.paged_decode(qg, kc, vc, table, lens, bs, 0.7)
+    kr = np.repeat(kc, G, axis=1)
+    vr = np.repeat(vc, G, axis=1)
+    O2, L2 = oracle.paged_decode(qg, kr, vr, table, lens, bs, 0.7)
+    np.testing.assert_array_equal(O, O2)
+    np.testing.assert_array_equal(L, L2)
+    with pytest.raises(ValueError):
+        oracle.paged_decode(qg[:, :5], kc, vc, table, lens, bs, 0.7)
