@@ -19,6 +19,7 @@ from .attention import (  # noqa: F401
     kv_append,
     merge_partials,
     paged_decode,
+    paged_prefill,
     scores,
     softmax_probs,
 )

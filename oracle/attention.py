@@ -317,3 +317,44 @@ def block_copy(k_cache, v_cache, src_blocks, dst_blocks):
         k_out[b] = k_cache[a]
         v_out[b] = v_cache[a]
     return k_out, v_out, skipped
+
+
+def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: int, scale: float, seqs=None):
+    """Multi-token paged prefill / append oracle.
+
+    [实现解析] §2.2 runs its paged loop "for each query position i"; [实现解析]
+    §2.3 and [区别] Q2 put PagedAttention's storage under FlashAttention's
+    computation.  Sequence s has n_s = cu_q[s+1] - cu_q[s] new query tokens,
+    the last n_s of its seq_lens[s] = L_s cached tokens (their keys/values
+    are already in the cache).  Query token i sits at position
+    L_s - n_s + i and attends keys 0 .. L_s - n_s + i (causal, offset by the
+    cached prefix).  Keys/values are resolved by explicit copy
+    (:func:`gather_paged`); query head h reads key/value head h // G
+    (G = Hq / Hkv).  q [total_q, Hq, d] -> O [total_q, Hq, d], LSE [total_q, Hq];
+    sequences not in ``seqs`` stay NaN.
+    """
+    T, H, d = q.shape
+    Hkv = k_cache.shape[1]
+    if H % Hkv:
+        raise ValueError("query heads must be a multiple of key/value heads")
+    G = H // Hkv
+    O = np.full((T, H, v_cache.shape[3]), np.nan)
+    LSE = np.full((T, H), np.nan)
+    S = len(seq_lens)
+    for s in (range(S) if seqs is None else seqs):
+        q0, q1 = int(cu_q[s]), int(cu_q[s + 1])
+        n, L = q1 - q0, int(seq_lens[s])
+        if n == 0:
+            continue
+        if n > L:
+            raise ValueError("a sequence has more new tokens than cached tokens")
+        Ks = gather_paged(k_cache, block_table[s], L, block_size)
+        Vs = gather_paged(v_cache, block_table[s], L, block_size)
+        for h in range(H):
+            for i in range(n):
+                p = L - n + i
+                o, lse = attention_head(np.asarray(q[q0 + i, h:h + 1], dtype=np.float64), Ks[h // G][:p + 1],
+                                        Vs[h // G][:p + 1], False, scale)
+                O[q0 + i, h] = o[0]
+                LSE[q0 + i, h] = lse[0]
+    return O, LSE

@@ -468,3 +468,41 @@ def test_paged_decode_grouped_query_heads():
     np.testing.assert_array_equal(L, L2)
     with pytest.raises(ValueError):
         oracle.paged_decode(qg[:, :5], kc, vc, table, lens, bs, 0.7)
+
+
+def test_paged_prefill_reduces_to_dense_causal_and_decode():
+    """Paged prefill pins: (1) a sequence whose every token is new is dense
+    causal attention on the gathered K/V (torch SDPA-pinned oracle); (2) one
+    new token per sequence is paged decode; (3) n new tokens of a longer
+    sequence equal the last n rows of dense causal attention over all L."""
+    rng = np.random.default_rng(70)
+    H, d, bs, nb = 2, 4, 4, 40
+    kc = rng.standard_normal((nb, H, bs, d))
+    vc = rng.standard_normal((nb, H, bs, d))
+    table = rng.permutation(nb)[:30].reshape(3, 10)
+    lens = np.array([13, 22, 9])
+    n_new = np.array([13, 1, 4])
+    cu = np.concatenate([[0], np.cumsum(n_new)])
+    q = rng.standard_normal((cu[-1], H, d))
+    O, L = oracle.paged_prefill(q, kc, vc, table, lens, cu, bs, 0.6)
+    for s in range(3):
+        Ks = oracle.gather_paged(kc, table[s], lens[s], bs)
+        Vs = oracle.gather_paged(vc, table[s], lens[s], bs)
+        for h in range(H):
+            # queries placed at the last n positions of a length-L causal problem
+            Qfull = np.zeros((lens[s], d))
+            Qfull[lens[s] - n_new[s]:] = q[cu[s]:cu[s + 1], h]
+            Od, Ld = A.attention_head(Qfull, Ks[h], Vs[h], True, 0.6)
+            np.testing.assert_allclose(O[cu[s]:cu[s + 1], h], Od[lens[s] - n_new[s]:], atol=1e-13)
+            np.testing.assert_allclose(L[cu[s]:cu[s + 1], h], Ld[lens[s] - n_new[s]:], atol=1e-13)
+    Od, Ld = oracle.paged_decode(q[cu[1]:cu[2]], kc, vc, table[1:2], lens[1:2], bs, 0.6)
+    np.testing.assert_allclose(O[cu[1]:cu[2]], Od, atol=1e-13)
+    # (4) grouped heads: query heads 2h, 2h+1 read key/value head h, the same as
+    # a multi-head cache holding each key/value head twice
+    qg = rng.standard_normal((cu[-1], 2 * H, d))
+    Og, Lg = oracle.paged_prefill(qg, kc, vc, table, lens, cu, bs, 0.6)
+    Om, Lm = oracle.paged_prefill(qg, np.repeat(kc, 2, axis=1), np.repeat(vc, 2, axis=1), table, lens, cu, bs, 0.6)
+    np.testing.assert_array_equal(Og, Om)
+    np.testing.assert_array_equal(Lg, Lm)
+    with pytest.raises(ValueError):
+        oracle.paged_prefill(q, kc, vc, table, np.array([13, 22, 3]), cu, bs, 0.6)  # 4 new tokens, 3 cached
