@@ -12,6 +12,8 @@ A step is one call of the entry point on one batch of the workload:
   decode_gqa_g4/_g8    paged_attn_decode_gqa, decode_uniform with 32 query heads over 8 / 4 K/V heads
   kv_append            paged_kv_append, 64 seqs x 512 new tokens (H=32, d=128, bs=16)
   block_copy           paged_block_copy, 1024 block pairs (copy-on-write), 128 KiB per block
+  prefill_paged_chunked paged_attn_prefill, 8 seqs x 2048 new tokens after U{0..6144} cached,
+                       32 query heads over 8 K/V heads, d=128, bs=16
 The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
 decode_uniform, measured the same way in the same run, under "decode".
 
@@ -520,6 +522,120 @@ class BlockCopy:
         return self.work * n / self.cfg["pairs"], dt, f"{n} of {self.cfg['pairs']} pairs"
 
 
+class PagedPrefill:
+    """paged_attn_prefill on the chunked-prefill workload.  Work = 4 * d *
+    H_q * (visible query-key pairs), new token i of sequence s seeing
+    ctx_s + i + 1 keys."""
+
+    def __init__(self, name, device, seed=0):
+        self.name = name
+        self.cfg = dict(W.PREFILL_PAGED_CHUNKED)
+        self.copies = 2
+        self.sets = [W.paged_chunked_prefill(device=device, seed=seed + 10 * i, **self.cfg)
+                     for i in range(self.copies)]
+        p = self.sets[0]
+        self.O = torch.empty_like(p.q)
+        self.LSE = torch.empty(p.q.shape[:2], dtype=torch.float32, device=device)
+        self.max_q = self.cfg["chunk"]
+        d, Hq = self.cfg["d"], self.cfg["Hq"]
+        pairs = []
+        for q in self.sets:
+            sl, n = q.seq_lens.cpu().tolist(), q.n_new.tolist()
+            pairs.append(sum(nn * (L - nn) + nn * (nn + 1) // 2 for L, nn in zip(sl, n)))
+        self.work_per_set = [4.0 * d * Hq * x for x in pairs]
+        self.work = statistics.mean(self.work_per_set)
+        self.unit, self.scale_unit = "TFLOP/s", 1e12
+        self.launches_per_step = 1
+        self.kernel = "prefill_bf16_kernel"
+
+    def step(self, i, osp):
+        p = self.sets[i % self.copies]
+        osp.paged_attn_prefill(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.cu_q, p.block_size,
+                               max_q_per_seq=self.max_q, O=self.O, LSE=self.LSE, scale=p.scale)
+
+    def config(self):
+        c = self.cfg
+        return {"workload": self.name, **c, "dtype": "bf16", "global_batch": c["num_seqs"], "seq_len": c["chunk"],
+                "flop_per_step": self.work,
+                "l2": f"inputs rotate over {self.copies} sets; K/V read per step ~{self._kv_mib():.0f} MiB > L2"}
+
+    def _kv_mib(self):
+        p = self.sets[0]
+        return float(p.seq_lens.sum()) * 2 * self.cfg["Hkv"] * self.cfg["d"] * 2 / 2**20
+
+    def e2e(self, osp, steps, device):
+        p = self.sets[0]
+        hq = p.q.cpu().pin_memory()
+        meta = [t.cpu().pin_memory() for t in (p.block_table, p.seq_lens, p.cu_q)]
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty(self.LSE.shape, dtype=torch.float32).pin_memory()
+        dq = torch.empty_like(p.q)
+        dmeta = [torch.empty_like(t) for t in (p.block_table, p.seq_lens, p.cu_q)]
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            dq.copy_(hq, non_blocking=True)
+            for d_, h_ in zip(dmeta, meta):
+                d_.copy_(h_, non_blocking=True)
+            osp.paged_attn_prefill(dq, p.k_cache, p.v_cache, dmeta[0], dmeta[1], dmeta[2], p.block_size,
+                                   max_q_per_seq=self.max_q, O=self.O, LSE=self.LSE, scale=p.scale)
+            ho.copy_(self.O, non_blocking=True)
+            hl.copy_(self.LSE, non_blocking=True)
+
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / steps
+        h2d = hq.numel() * 2 + sum(t.numel() * 4 for t in meta)
+        d2h = ho.numel() * 2 + hl.numel() * 4
+        return ms * self.work / self.work_per_set[0], h2d, d2h
+
+    def oracle_rows(self, s, h, rows):
+        """The oracle on given new-token rows of (sequence s, query head h);
+        returns the FLOPs those rows stand for."""
+        import numpy as np
+        import oracle
+        p = self.sets[0]
+        L = int(p.seq_lens[s])
+        n = int(p.cu_q[s + 1] - p.cu_q[s])
+        q0 = int(p.cu_q[s])
+        G = self.cfg["Hq"] // self.cfg["Hkv"]
+
+        class Lazy:
+            def __init__(self, t):
+                self.t, self.shape = t, tuple(t.shape)
+
+            def __getitem__(self, i):
+                return self.t[int(i)].double().cpu().numpy()
+
+        tbl = p.block_table[s].cpu().numpy()
+        K = oracle.gather_paged(Lazy(p.k_cache), tbl, L, p.block_size)[h // G]
+        V = oracle.gather_paged(Lazy(p.v_cache), tbl, L, p.block_size)[h // G]
+        work = 0.0
+        for i in rows:
+            pos = L - n + i
+            q = p.q[q0 + i, h:h + 1].double().cpu().numpy()
+            oracle.attention_head(q, K[:pos + 1], V[:pos + 1], False, p.scale)
+            work += 4.0 * self.cfg["d"] * (pos + 1)
+        return work
+
+    def cpu_sample(self, budget_s):
+        """The oracle on rows of (sequence 0, head 0), 64 at a time, until the budget."""
+        t0 = time.perf_counter()
+        work, done = 0.0, 0
+        while time.perf_counter() - t0 < budget_s and done < self.cfg["chunk"]:
+            work += self.oracle_rows(0, 0, range(done, min(done + 64, self.cfg["chunk"])))
+            done = min(done + 64, self.cfg["chunk"])
+        dt = time.perf_counter() - t0
+        return work, dt, f"new-token rows 0..{done - 1} of sequence 0, query head 0 (K/V gathered per 64 rows)"
+
+
 def make_workload(name, device, seed=0):
     if name == "prefill_2k":
         return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
@@ -531,6 +647,8 @@ def make_workload(name, device, seed=0):
         return KVAppend(name, device, seed)
     if name == "block_copy":
         return BlockCopy(name, device, seed)
+    if name == "prefill_paged_chunked":
+        return PagedPrefill(name, device, seed)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -612,7 +730,7 @@ def run_ours(args):
     pk, pk_src = peaks()
 
     wl = make_workload(args.workload, device, seed=args.seed + rank)
-    bound = "tensor" if isinstance(wl, Prefill) else "hbm"
+    bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill)) else "hbm"
     with ClockSampler(local) as clocks:
         t_load0 = time.perf_counter()
         per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak)
@@ -683,7 +801,18 @@ def run_reference(args):
     import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     name = args.workload
-    if name.startswith("prefill"):
+    if name == "prefill_paged_chunked":
+        wl = PagedPrefill(name, dev, args.seed)
+        unit, su = "TFLOP/s", 1e12
+        S = wl.cfg["num_seqs"]
+
+        def one(i):
+            s, h = i % S, (7 * i) % wl.cfg["Hq"]
+            return wl.oracle_rows(s, h, range(0, wl.cfg["chunk"], 128))
+
+        sample = f"16 new-token rows of one (sequence, head) of {name} per step"
+        config = wl.config()
+    elif name.startswith("prefill"):
         cfg = W.PREFILL_CAUSAL_2K if name == "prefill_2k" else W.PREFILL_CAUSAL_16K
         B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
         pairs = N * (N + 1) // 2
@@ -752,7 +881,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_2k",
                     choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
-                             "decode_uniform_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8"])
+                             "decode_uniform_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8",
+                             "prefill_paged_chunked"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")

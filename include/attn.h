@@ -162,6 +162,45 @@ ATTN_API attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, c
                                            attn_stream_t stream);
 
 /*
+ * Multi-token paged prefill (chunked prefill / prefix reuse): several new
+ * query tokens per sequence attend causally to that sequence's paged cache,
+ * which already holds their own keys and values ("第 2 章核心模块：
+ * FlashAttention-2 与 PagedAttention 实现解析" section 2.2 runs the paged loop
+ * for each query position; section 2.3 pairs PagedAttention's storage with
+ * FlashAttention's tiled computation).
+ *
+ * q, O         : [total_q, H_q, d] bf16, the new tokens of all sequences
+ *                packed: sequence s owns rows cu_q[s] .. cu_q[s+1]-1.
+ * LSE          : [total_q, H_q] fp32.
+ * cu_q         : int32 [num_seqs + 1], cu_q[0] = 0, non-decreasing.
+ * seq_lens     : int32 [num_seqs], keys cached for each sequence including
+ *                its n_s = cu_q[s+1] - cu_q[s] new tokens; new token i of
+ *                sequence s is at position seq_lens[s] - n_s + i and sees
+ *                keys 0 .. that position.
+ * block_table,
+ * caches       : as for paged_attn_decode_gqa (H_kv key/value heads; query
+ *                head h reads key/value head h / (H_q / H_kv)).
+ * max_q_per_seq: an upper bound of n_s (host value; sizes the work grid).
+ * Supported    : bf16; d in {64, 128}; block_size in {16, 32}.  Runs on the
+ *                tcgen05 prefill kernel, one TMA box per cache block.
+ * Device checks: a table entry outside [0, num_blocks) sets
+ *                ATTN_DEVERR_BLOCK_TABLE (block 0 is read in its place and the
+ *                sequence's rows are not meaningful); cu_q entries outside
+ *                [0, total_q] or decreasing set ATTN_DEVERR_INDEX; a sequence
+ *                with n_s > seq_lens[s] or seq_lens[s] > max_blocks_per_seq *
+ *                block_size sets ATTN_DEVERR_SEQ_LEN.  The rows of a sequence
+ *                flagged by either of the last two are not written.
+ * Cache slots past seq_lens[s] may hold any bits (NaN included): they take
+ *                no part in the product.
+ */
+ATTN_API attn_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                        const int32_t *block_table, const int32_t *seq_lens, const int32_t *cu_q,
+                                        int block_size, void *O, float *LSE, int num_seqs, int total_q,
+                                        int max_q_per_seq, int H_q, int H_kv, int d, int num_blocks,
+                                        int max_blocks_per_seq, float scale, attn_dtype dt, int32_t *err_flag,
+                                        attn_stream_t stream);
+
+/*
  * Paged decode without a workspace argument, for callers that cannot
  * allocate device memory (code running where cudaMalloc is not permitted or
  * not wanted, e.g. inside an allocator or pool callback, in a process whose

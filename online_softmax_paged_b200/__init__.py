@@ -17,7 +17,7 @@ __all__ = [
     "AttnError", "attn_fwd", "paged_attn_decode", "paged_attn_decode_workspace_size",
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
-    "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa",
+    "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,8 @@ ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_I
 
 # every function include/attn.h declares
 EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
-                    "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_kv_append",
+                    "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_attn_prefill",
+                    "paged_kv_append",
                     "paged_block_copy",
                     "attn_read_error", "attn_status_str")
 
@@ -74,6 +75,9 @@ def load():
     lib.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                               c_float, c_int, vp, vp]
     lib.paged_attn_decode_noalloc.restype = c_int
+    lib.paged_attn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
+                                       c_int, c_int, c_int, c_float, c_int, vp, vp]
+    lib.paged_attn_prefill.restype = c_int
     lib.paged_kv_append.argtypes = [vp, vp, vp, vp, c_int, vp, c_int, c_int, vp, vp, c_int, c_int, c_int, c_int,
                                     c_int, vp, vp]
     lib.paged_kv_append.restype = c_int
@@ -213,6 +217,44 @@ def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size
                                       _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode_gqa")
+    return O, LSE
+
+
+def paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size, max_q_per_seq=None, O=None,
+                       LSE=None, scale=None, err_flag=None, stream=None):
+    """Multi-token paged prefill: q [total_q, H_q, d] bf16 packed by cu_q
+    (int32 [S + 1]); caches [num_blocks, H_kv, block_size, d] already holding
+    the new tokens' keys/values; seq_lens counts them.  ``max_q_per_seq`` is
+    read from cu_q (one device-to-host copy) when not given.  See
+    include/attn.h."""
+    _check_cuda(q, k_cache, v_cache, block_table, seq_lens, cu_q, O, LSE, err_flag)
+    T, Hq, d = q.shape
+    nb, Hkv, bs, dk = k_cache.shape
+    S = seq_lens.shape[0]
+    for t in (block_table, seq_lens, cu_q):
+        if t.dtype != torch.int32:
+            raise ValueError("block_table, seq_lens and cu_q must be int32")
+    if cu_q.shape != (S + 1,) or block_table.shape[0] != S:
+        raise ValueError("cu_q must be [S + 1] and block_table [S, max_blocks]")
+    if k_cache.shape != v_cache.shape or bs != block_size or dk != d:
+        raise ValueError("caches must be [num_blocks, H_kv, block_size, d]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens, cu_q):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if max_q_per_seq is None:
+        max_q_per_seq = int((cu_q[1:] - cu_q[:-1]).max().item()) if S > 0 else 0
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = load().paged_attn_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                   _ptr(cu_q), int(block_size), _ptr(O), _ptr(LSE), S, T, int(max_q_per_seq), Hq,
+                                   Hkv, d, nb, block_table.shape[1], float(scale), _dtype_code(q.dtype),
+                                   _ptr(err_flag), _stream(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_attn_prefill")
     return O, LSE
 
 

@@ -94,6 +94,35 @@ attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, const void
                        num_blocks, max_blocks_per_seq, scale, dt, workspace, workspace_bytes, err_flag, stream);
 }
 
+attn_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                               const int32_t *seq_lens, const int32_t *cu_q, int block_size, void *O, float *LSE,
+                               int num_seqs, int total_q, int max_q_per_seq, int H_q, int H_kv, int d, int num_blocks,
+                               int max_blocks_per_seq, float scale, attn_dtype dt, int32_t *err_flag,
+                               attn_stream_t stream) {
+    if (dt != ATTN_F32 && dt != ATTN_BF16) return ATTN_EINVAL;
+    if (num_seqs < 0 || total_q < 0 || max_q_per_seq < 0 || H_q < 1 || H_kv < 1 || num_blocks < 1 ||
+        max_blocks_per_seq < 1)
+        return ATTN_EINVAL;
+    if (H_q % H_kv) return ATTN_EINVAL;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
+    if (dt != ATTN_BF16) return ATTN_EUNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return ATTN_EUNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return ATTN_EINVAL;
+    if ((long long)num_blocks * H_kv * block_size > 0x7fffffffLL) return ATTN_EINVAL;
+    if ((long long)total_q * H_q > 0x7fffffffLL || (long long)num_seqs * H_q > 0x7fffffffLL / 64) return ATTN_EINVAL;
+    if (num_seqs == 0 || total_q == 0 || max_q_per_seq == 0) return ATTN_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !cu_q || !O || !LSE) return ATTN_EINVAL;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(O)) return ATTN_EINVAL;
+    if (((uintptr_t)block_table & 3u) || ((uintptr_t)seq_lens & 3u) || ((uintptr_t)cu_q & 3u) ||
+        ((uintptr_t)LSE & 3u))
+        return ATTN_EINVAL;
+    osp::PagedPrefillLaunch p{q,       k_cache, v_cache, block_table, seq_lens,   cu_q,               O,
+                              LSE,     num_seqs, total_q, max_q_per_seq, H_q,      H_kv,              d,
+                              num_blocks, max_blocks_per_seq, block_size, scale,   err_flag};
+    return osp::launch_paged_prefill(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 attn_status paged_kv_append(const void *k_new, const void *v_new, const int32_t *seq_ids, const int32_t *positions,
                             int num_tokens, const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
                             void *k_cache, void *v_cache, int num_blocks, int H, int d, int block_size,

@@ -47,7 +47,18 @@ struct CopyLaunch {
     int32_t *err_flag;
 };
 
+struct PagedPrefillLaunch {
+    const void *q, *k_cache, *v_cache;
+    const int32_t *block_table, *seq_lens, *cu_q;
+    void *O;
+    float *LSE;
+    int num_seqs, total_q, max_q_per_seq, Hq, Hkv, d, num_blocks, max_blocks, block_size;
+    float scale;
+    int32_t *err_flag;
+};
+
 attn_status launch_dense_f32(const DenseLaunch &p, cudaStream_t stream);
+attn_status launch_paged_prefill(const PagedPrefillLaunch &p, cudaStream_t stream);
 attn_status launch_kv_append(const AppendLaunch &p, cudaStream_t stream);
 attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream);
 attn_status launch_prefill_bf16(const DenseLaunch &p, cudaStream_t stream);

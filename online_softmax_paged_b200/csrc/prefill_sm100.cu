@@ -78,6 +78,20 @@ struct PrefillArgs {
     int32_t *err;
     int N, BH, nblk;
     float scale_log2;
+    // paged mode: query tokens of sequence s are rows cu_q[s] .. cu_q[s+1]-1 of
+    // q / O / LSE, at key positions seq_lens[s] - n_s .. seq_lens[s] - 1
+    const int32_t *cu_q, *seq_lens, *block_table;
+    int S, Hq, Hkv, max_blocks, num_blocks, block_size, nqb, total_q;
+};
+
+// What every role needs to know about a work unit (256 query rows of one
+// head).  Dense: rows qrow0 .. of head `head` ((b, h) flattened), keys 0 .. N-1.
+// Paged: rows qrow0 .. of sequence s's new tokens, query head `head`,
+// key/value head kv_head, keys 0 .. L-1, row r at key position pos0 + r.
+struct UnitInfo {
+    int head, kv_head, s, qrow0, nq, pos0, L, qtok0;
+    int n0, n1;  // key tiles of query tile 0 / 1 (0: the tile has no rows)
+    int bad;     // paged: device error bits of an inconsistent sequence (0: fine)
 };
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -224,15 +238,52 @@ __device__ __forceinline__ int snake_unit(int r, int c, int G, int n_units) {
     return u < n_units ? u : -1;
 }
 
-// Key tiles each query tile of unit (blk) visits; 0 when the tile is past N.
-__device__ __forceinline__ void tile_counts(const PrefillArgs &a, bool causal, int blk, int &n0, int &n1) {
-    const int n_kv_all = (a.N + BN - 1) / BN;
-    const int q0 = NQ * blk, q1 = NQ * blk + 1;
-    n0 = (q0 * BM >= a.N) ? 0 : (causal ? min(q0 + 1, n_kv_all) : n_kv_all);
-    n1 = (q1 * BM >= a.N) ? 0 : (causal ? min(q1 + 1, n_kv_all) : n_kv_all);
+// Unit u of the kernel's unit space -> UnitInfo.  Dense units are numbered
+// longest first when causal; paged units as (query block, sequence, head)
+// with later query blocks (more keys) first.  A paged unit past its
+// sequence's new tokens, or of an inconsistent sequence, gets n0 = n1 = 0;
+// the latter also gets `bad` (cu_q outside [0, total_q] or decreasing:
+// ATTN_DEVERR_INDEX; more new tokens than cached keys, or more keys than the
+// table holds: ATTN_DEVERR_SEQ_LEN).
+template <bool PAGED>
+__device__ __forceinline__ void get_unit(const PrefillArgs &a, bool causal, int u, UnitInfo &x) {
+    x.bad = 0;
+    if (!PAGED) {
+        int blk;
+        unit_coords(a, causal, u, blk, x.head);
+        x.kv_head = x.head;
+        x.s = 0;
+        x.qrow0 = NQ * BM * blk;
+        x.nq = x.L = a.N;
+        x.pos0 = 0;
+        x.qtok0 = 0;
+    } else {
+        const int SH = a.S * a.Hq;
+        const int qb = a.nqb - 1 - u / SH, rem = u % SH;
+        x.s = rem / a.Hq;
+        x.head = rem - x.s * a.Hq;
+        x.kv_head = x.head / (a.Hq / a.Hkv);
+        x.qtok0 = a.cu_q[x.s];
+        x.nq = a.cu_q[x.s + 1] - x.qtok0;
+        x.L = a.seq_lens[x.s];
+        x.pos0 = x.L - x.nq;
+        x.qrow0 = NQ * BM * qb;
+        if (x.qtok0 < 0 || x.nq < 0 || x.qtok0 + x.nq > a.total_q) x.bad = ATTN_DEVERR_INDEX;
+        else if (x.pos0 < 0 || (long long)x.L > (long long)a.max_blocks * a.block_size) x.bad = ATTN_DEVERR_SEQ_LEN;
+    }
+    const int n_kv_all = (x.L + BN - 1) / BN;
+    int n[NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        const int r0 = x.qrow0 + i * BM;
+        n[i] = (x.bad || r0 >= x.nq) ? 0
+               : (causal ? min((x.pos0 + r0 + BM - 1) / BN + 1, n_kv_all) : n_kv_all);
+    }
+    x.n0 = n[0];
+    x.n1 = n[1];
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
@@ -253,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
-    const int n_units = a.nblk * a.BH;
+    const int n_units = PAGED ? a.nqb * a.S * a.Hq : a.nblk * a.BH;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -296,9 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = snake_unit(r, c, G, n_units);
                 if (u < 0) break;
-                int blk, bh, n0, n1;
-                unit_coords(a, CAUSAL, u, blk, bh);
-                tile_counts(a, CAUSAL, blk, n0, n1);
+                UnitInfo x;
+                get_unit<PAGED>(a, CAUSAL, u, x);
+                const int n0 = x.n0, n1 = x.n1;
+                if (PAGED && x.bad && x.qrow0 == 0 && x.head == 0 && elect_one() && a.err)
+                    atomicOr(a.err, x.bad);
                 for (int i = 0; i < NQ && ok; ++i) {
                     if ((i ? n1 : n0) == 0) continue;
                     // the previous unit's QK^T products of this tile are done
@@ -307,8 +360,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
                     if (elect_one()) {
                         mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b)
-                            tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, (NQ * blk + i) * BM, bh);
+                        for (int b = 0; b < C::kBoxes; ++b) {
+                            if (PAGED)  // rows past the sequence's tokens are loaded but never stored
+                                tma_load_2d(dst + b * kBoxBytes, &tmQ, &q_full[i], x.head * D + b * kBoxCols,
+                                            x.qtok0 + x.qrow0 + i * BM);
+                            else
+                                tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, x.qrow0 + i * BM,
+                                            x.head);
+                        }
                     }
                     ++qc[i];
                 }
@@ -320,10 +379,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     const CUtensorMap *tm = (v & 1) ? &tmV : &tmK;
                     uint8_t *dst = smem + C::kRingOff + slot * C::kTileBytes;
-                    if (elect_one()) {
-                        mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b)
-                            tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN, bh);
+                    if (!PAGED) {
+                        if (elect_one()) {
+                            mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+                            for (int b = 0; b < C::kBoxes; ++b)
+                                tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN,
+                                            x.head);
+                        }
+                    } else {
+                        // one box per cache block: lane k loads block k of the tile.
+                        // Blocks past the sequence load its block 0 instead (finite
+                        // data under masked keys); ids outside the pool use block 0
+                        // and are reported.
+                        const int per = BN / a.block_size;
+                        const int lb0 = (v >> 1) * per;
+                        const int nblk_seq = (x.L + a.block_size - 1) / a.block_size;
+                        int phys = 0;
+                        if (lane < per) {
+                            const int32_t *row = a.block_table + (size_t)x.s * a.max_blocks;
+                            phys = row[lb0 + lane < nblk_seq ? lb0 + lane : 0];
+                            if (phys < 0 || phys >= a.num_blocks) {
+                                if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+                                phys = 0;
+                            }
+                        }
+                        if (elect_one()) mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+                        __syncwarp();
+                        if (lane < per) {
+                            const int y = (phys * a.Hkv + x.kv_head) * a.block_size;
+                            for (int b = 0; b < C::kBoxes; ++b)
+                                tma_load_2d(dst + b * kBoxBytes + lane * a.block_size * 128, tm, &kv_full[slot],
+                                            b * kBoxCols, y);
+                        }
+                        __syncwarp();
                     }
                 }
             }
@@ -360,7 +448,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_s = [&](int i, uint32_t u) {
                 const uint64_t da = i ? dq1 : dq0, db = dk + slot_off(u);
                 const uint32_t d_tm = i ? tm_s1 : tm_s0;
-#pragma unroll
                 if (elect_one()) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
@@ -371,12 +458,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             };
-            auto issue_pv = [&](int i, uint32_t u, int j) {
+            // nks: 16-key steps of the tile that hold live keys (BN / 16 but for
+            // a paged sequence's last tile)
+            auto issue_pv = [&](int i, uint32_t u, int j, int nks) {
                 const uint64_t db = dv + slot_off(u);
                 const uint32_t d_tm = i ? tm_o1 : tm_o0, p_tm = i ? tm_s1 : tm_s0;
                 if (elect_one()) {
 #pragma unroll
                     for (int ks = 0; ks < BN / 16; ++ks)
+                        if (ks < nks)
                         mma_ts(d_tm, p_tm + ks * 8, db + (uint64_t)((ks * 16 * 128) >> 4), idesc_pv,
                                (j > 0 || ks > 0));
                     mma_commit(&o_full[i]);
@@ -386,10 +476,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = snake_unit(r, c, G, n_units);
                 if (u < 0) break;
-                int blk, bh, n0, n1;
-                unit_coords(a, CAUSAL, u, blk, bh);
-                tile_counts(a, CAUSAL, blk, n0, n1);
+                UnitInfo x;
+                get_unit<PAGED>(a, CAUSAL, u, x);
+                const int n0 = x.n0, n1 = x.n1;
                 const int nkv_max = max(n0, n1);
+                if (nkv_max == 0) continue;  // a paged unit with no rows
                 if (n0 > 0) ok = wait_or_abort(&q_full[0], qc0 & 1, a.err, abort_flag);
                 if (ok && n1 > 0) ok = wait_or_abort(&q_full[1], qc1 & 1, a.err, abort_flag);
                 if (ok) ok = wait_kv(ukv);
@@ -403,10 +494,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n0 == 1) mma_commit(&q_empty[0]);
                     if (n1 == 1) mma_commit(&q_empty[1]);
                 }
+                const int n_kv_all = (x.L + BN - 1) / BN;
                 for (int j = 0; j < nkv_max && ok; ++j) {
                     const uint32_t uV = ukv + 2 * j + 1, uK = ukv + 2 * j + 2;
                     ok = wait_kv(uV);
                     if (!ok) break;
+                    int nks = BN / 16;
+                    if (PAGED && j == n_kv_all - 1) {
+                        // A paged sequence's last tile: cache slots past its end hold
+                        // whatever the pool holds (NaN included) and 0 * NaN = NaN in
+                        // P.V.  Issue only the 16-key steps with live keys and zero
+                        // the dead V rows of the last one (masked P is ~0 there).
+                        const int live = x.L - j * BN;
+                        nks = (live + 15) >> 4;
+                        const int dead = nks * 16 - live;  // rows live .. 16 * nks - 1
+                        uint8_t *vslot = smem + C::kRingOff + (uV % C::kStages) * C::kTileBytes;
+                        for (int t = lane; t < dead * 8 * C::kBoxes; t += 32) {
+                            const int b = t / (dead * 8), rem = t - b * dead * 8;
+                            *reinterpret_cast<uint4 *>(vslot + b * kBoxBytes + (live + rem / 8) * 128 + (rem % 8) * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
                     bool k_ready = false;
 #pragma unroll
                     for (int i = 0; i < NQ; ++i) {
@@ -415,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = wait_or_abort(&p_full[i], ((i ? it1 : it0) + j) & 1, a.err, abort_flag);
                         if (!ok) continue;
                         tc_fence_after();
-                        issue_pv(i, uV, j);
+                        issue_pv(i, uV, j, nks);
                         if (j + 1 < ni) {
                             if (!k_ready) {
                                 ok = wait_kv(uK);
@@ -468,12 +578,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int rr = 0; ok; ++rr) {
             const int u = snake_unit(rr, c, G, n_units);
             if (u < 0) break;
-            int blk, bh, n0, n1;
-            unit_coords(a, CAUSAL, u, blk, bh);
-            tile_counts(a, CAUSAL, blk, n0, n1);
-            const int my_nkv = i ? n1 : n0;
-            const int qt = NQ * blk + i;
-            const int row = qt * BM + r_in;      // query row in the sequence
+            UnitInfo x;
+            get_unit<PAGED>(a, CAUSAL, u, x);
+            const int my_nkv = i ? x.n1 : x.n0;
+            const int tile_pos = x.pos0 + x.qrow0 + i * BM;  // key position of the tile's row 0
+            const int row = x.qrow0 + i * BM + r_in;        // query row in the sequence
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < my_nkv; ++j) {
                 ok = wait_or_abort(&s_full[i], (itc + j) & 1, a.err, abort_flag);
@@ -483,13 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_tm + 32 * cc, sr[cc]);
                 tmem_wait_ld();
-                // visible keys: col <= lim; only the causal diagonal tile and the
+                // visible keys: col <= lim; only key tiles reaching past the
+                // tile's first row position (the causal diagonal) and the
                 // sequence's last tile need masking
-                const bool masked = (CAUSAL && j == qt) || ((j + 1) * BN > a.N);
+                const bool masked = (CAUSAL && (j + 1) * BN - 1 > tile_pos) || ((j + 1) * BN > x.L);
                 if (masked) {
                     int lim = BN - 1;
-                    if (CAUSAL && j == qt) lim = r_in;
-                    lim = min(lim, a.N - 1 - j * BN);
+                    if (CAUSAL) lim = min(lim, tile_pos + r_in - j * BN);
+                    lim = min(lim, x.L - 1 - j * BN);
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
@@ -558,8 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                const bool live = row < a.N;
-                __nv_bfloat16 *orow = a.O + ((size_t)bh * a.N + (live ? row : 0)) * D;
+                const bool live = row < x.nq;
+                const size_t orow_idx = PAGED ? ((size_t)(x.qtok0 + (live ? row : 0)) * a.Hq + x.head)
+                                              : ((size_t)x.head * a.N + (live ? row : 0));
+                __nv_bfloat16 *orow = a.O + orow_idx * D;
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t orr[32];
@@ -576,8 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
                 }
-                if (live)
-                    a.LSE[(size_t)bh * a.N + row] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+                if (live) a.LSE[orow_idx] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
                 // the O reads are complete before the next unit's first PV may
                 // overwrite O (ordered through p_full of that unit)
                 tc_fence_before();
@@ -626,6 +737,21 @@ bool make_map(CUtensorMap *m, const void *base, int N, int d, int BH) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor map: `rows` rows of `inner` elements (row pitch
+// `pitch_elems`), box 64 x box_rows, 128B swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, long long inner, long long rows, long long pitch_elems,
+                 int box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)pitch_elems * 2};
+    cuuint32_t box[2] = {kBoxCols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, bool CAUSAL>
 attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
     using C = Cfg<D>;
@@ -633,7 +759,7 @@ attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ECUDA;
     if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(prefill_bf16_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(prefill_bf16_kernel<D, CAUSAL, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess)
             return ATTN_ECUDA;
         attr_set[dev] = true;
@@ -658,11 +784,60 @@ attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
     // each walking its units in snake order
     const long long units = (long long)a.nblk * BH;
     const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
-    prefill_bf16_kernel<D, CAUSAL><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+    prefill_bf16_kernel<D, CAUSAL, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+template <int D>
+attn_status launch_paged_t(const PagedPrefillLaunch &p, cudaStream_t stream) {
+    using C = Cfg<D>;
+    static bool attr_set[64] = {false};
+    static int sm_count[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ECUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(prefill_bf16_kernel<D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return ATTN_ECUDA;
+        attr_set[dev] = true;
+    }
+    if (sm_count[dev] == 0 &&
+        cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ECUDA;
+    CUtensorMap tq, tk, tv;
+    const long long cache_rows = (long long)p.num_blocks * p.Hkv * p.block_size;
+    if (!make_map_2d(&tq, p.q, (long long)p.Hq * D, p.total_q, (long long)p.Hq * D, BM) ||
+        !make_map_2d(&tk, p.k_cache, D, cache_rows, D, p.block_size) ||
+        !make_map_2d(&tv, p.v_cache, D, cache_rows, D, p.block_size))
+        return ATTN_ECUDA;
+    PrefillArgs a = {};
+    a.O = static_cast<__nv_bfloat16 *>(p.O);
+    a.LSE = p.LSE;
+    a.err = p.err_flag;
+    a.scale_log2 = p.scale * 1.4426950408889634f;
+    a.cu_q = p.cu_q;
+    a.seq_lens = p.seq_lens;
+    a.block_table = p.block_table;
+    a.S = p.num_seqs;
+    a.Hq = p.Hq;
+    a.Hkv = p.Hkv;
+    a.max_blocks = p.max_blocks;
+    a.num_blocks = p.num_blocks;
+    a.block_size = p.block_size;
+    a.nqb = (p.max_q_per_seq + NQ * BM - 1) / (NQ * BM);
+    a.total_q = p.total_q;
+    const long long units = (long long)a.nqb * a.S * a.Hq;
+    if (units == 0) return ATTN_OK;
+    const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
+    prefill_bf16_kernel<D, true, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
 }  // namespace
+
+attn_status launch_paged_prefill(const PagedPrefillLaunch &p, cudaStream_t stream) {
+    return p.d == 128 ? launch_paged_t<128>(p, stream) : launch_paged_t<64>(p, stream);
+}
 
 attn_status launch_prefill_bf16(const DenseLaunch &p, cudaStream_t stream) {
     if (p.d == 128) return p.causal ? launch_t<128, true>(p, stream) : launch_t<128, false>(p, stream);

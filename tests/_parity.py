@@ -33,3 +33,16 @@ def check_close(O_gpu, LSE_gpu, O_ref, LSE_ref, dtype, what=""):
         assert dO.mean() <= BF16_MEAN, f"{what}: mean|dO| {dO.mean():.3e} > {BF16_MEAN}"
     assert dL.max() <= LSE_MAX, f"{what}: max|dLSE| {dL.max():.3e} > {LSE_MAX}"
     return float(dO.max()), float(dO.mean()), float(dL.max())
+
+
+class DeviceCache:
+    """Host view of a device KV cache [num_blocks, H, block_size, d] that
+    copies one physical block (as float64) on access, so the oracle can
+    resolve a block table against a large device pool."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, i):
+        return self.t[int(i)].double().cpu().numpy()

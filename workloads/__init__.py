@@ -29,6 +29,11 @@ PREFILL_CAUSAL_16K = dict(B=1, H=32, N=16384, d=128, causal=True, dtype=torch.bf
 DECODE_UNIFORM = dict(num_seqs=64, H=32, d=128, block_size=16, pool=20000, len_lo=128, len_hi=4096)
 DECODE_SHARED_PREFIX = dict(num_seqs=256, H=32, d=128, block_size=32, pool=20000, median=1024,
                             sigma=1.0, len_lo=1, len_hi=8192, group=8, prefix_tokens=512)
+# chunked prefill over a paged cache: each sequence appends a 2048-token
+# chunk after a cached context of U{0..6144} tokens; 32 query heads over 8
+# key/value heads
+PREFILL_PAGED_CHUNKED = dict(num_seqs=8, Hq=32, Hkv=8, d=128, block_size=16, pool=20000, chunk=2048,
+                             ctx_lo=0, ctx_hi=6144)
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -188,6 +193,78 @@ def paged_shared_prefix(num_seqs=256, H=32, d=128, block_size=32, pool=20000, me
     q = _normal((num_seqs, H, d), g, device, dtype)
     return PagedInputs(q, k_cache, v_cache, table.to(device), seq_lens.to(torch.int32).to(device),
                        block_size, 1.0 / math.sqrt(d), groups)
+
+
+@dataclass
+class PagedPrefillInputs:
+    q: torch.Tensor            # [total_q, Hq, d], sequence s owns rows cu_q[s] .. cu_q[s+1]-1
+    k_cache: torch.Tensor      # [num_blocks, Hkv, block_size, d] (new tokens' keys included)
+    v_cache: torch.Tensor
+    block_table: torch.Tensor  # int32 [S, max_blocks_per_seq], unused entries -1
+    seq_lens: torch.Tensor     # int32 [S], cached context + new tokens
+    cu_q: torch.Tensor         # int32 [S + 1]
+    block_size: int
+    scale: float
+
+    @property
+    def num_seqs(self):
+        return self.seq_lens.shape[0]
+
+    @property
+    def n_new(self):
+        return (self.cu_q[1:] - self.cu_q[:-1]).cpu()
+
+    def shuffled(self, seed=1):
+        sh = shuffle_placement(PagedInputs(self.q, self.k_cache, self.v_cache, self.block_table, self.seq_lens,
+                                           self.block_size, self.scale), seed=seed)
+        return PagedPrefillInputs(self.q, sh.k_cache, sh.v_cache, sh.block_table, self.seq_lens, self.cu_q,
+                                  self.block_size, self.scale)
+
+
+def paged_prefill_inputs(ctx_lens, n_new, Hq=8, Hkv=8, d=128, block_size=16, pool=None, seed=0, device="cpu",
+                         dtype=torch.bfloat16, max_blocks_per_seq=None):
+    """Multi-token paged prefill inputs with given per-sequence cached context
+    lengths and new-token counts (seq_lens = ctx + n).
+
+    Draw order: one randperm(pool), sliced consecutively into each sequence's
+    ceil(seq_len / block_size) blocks (no block used twice); K cache; V cache
+    (N(0,1), every slot of the pool drawn, the new tokens' keys/values
+    included); q [sum n, Hq, d].  Unused table entries are -1.
+    """
+    ctx_lens, n_new = [int(x) for x in ctx_lens], [int(x) for x in n_new]
+    S = len(ctx_lens)
+    lens = [c + n for c, n in zip(ctx_lens, n_new)]
+    nbs = [-(-L // block_size) for L in lens]
+    pool = pool or max(1, sum(nbs) + 2)
+    g = _gen(seed, device)
+    perm = torch.randperm(pool, generator=g, device=device).cpu()
+    mb = max_blocks_per_seq or max(1, max(nbs) if nbs else 1)
+    table = torch.full((S, mb), -1, dtype=torch.int32)
+    cur = 0
+    for s in range(S):
+        if cur + nbs[s] > pool:
+            raise ValueError("pool too small for the given lengths")
+        table[s, :nbs[s]] = perm[cur:cur + nbs[s]].to(torch.int32)
+        cur += nbs[s]
+    k_cache = _cache(pool, Hkv, block_size, d, g, device, dtype)
+    v_cache = _cache(pool, Hkv, block_size, d, g, device, dtype)
+    cu = [0]
+    for n in n_new:
+        cu.append(cu[-1] + n)
+    q = _normal((cu[-1], Hq, d), g, device, dtype, 1.0, max(1, (1 << 26) // (Hq * d)))
+    return PagedPrefillInputs(q, k_cache, v_cache, table.to(device), torch.tensor(lens, dtype=torch.int32).to(device),
+                              torch.tensor(cu, dtype=torch.int32).to(device), block_size, 1.0 / math.sqrt(d))
+
+
+def paged_chunked_prefill(num_seqs=8, Hq=32, Hkv=8, d=128, block_size=16, pool=20000, chunk=2048, ctx_lo=0,
+                          ctx_hi=6144, seed=0, device="cpu", dtype=torch.bfloat16):
+    """Chunked-prefill workload: cached contexts ~ U{ctx_lo..ctx_hi} (drawn
+    first, from the same generator seed + 1), then :func:`paged_prefill_inputs`
+    with ``chunk`` new tokens per sequence."""
+    gc = _gen(seed + 1, "cpu")
+    ctx = torch.randint(ctx_lo, ctx_hi + 1, (num_seqs,), generator=gc).tolist()
+    mb = -(-(ctx_hi + chunk) // block_size)
+    return paged_prefill_inputs(ctx, [chunk] * num_seqs, Hq, Hkv, d, block_size, pool, seed, device, dtype, mb)
 
 
 def shuffle_placement(inp: PagedInputs, seed=1, pool=None) -> PagedInputs:
