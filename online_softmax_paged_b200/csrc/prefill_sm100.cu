@@ -65,11 +65,15 @@ struct Cfg {
     static constexpr int kStages = D == 128 ? 4 : 8;
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = NQ * kTileBytes;
-    static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], done
-    static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 1;
+    // one 64-column O box per query tile, staged for the TMA store
+    static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
+    static constexpr int kBarOff = kStageOff + NQ * kBoxBytes;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], done,
+    // stg_full[2], stg_free[2]
+    static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 1 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
 struct PrefillArgs {
@@ -286,7 +290,8 @@ __device__ __forceinline__ void get_unit(const PrefillArgs &a, bool causal, int 
 template <int D, bool CAUSAL, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                        PrefillArgs a) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -299,6 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *p_full = s_full + 2;
     uint64_t *o_full = p_full + 2;
     uint64_t *done_bar = o_full + 2;
+    uint64_t *stg_full = done_bar + 1;  // the tile's 128 rows are in its staging box
+    uint64_t *stg_free = stg_full + 2;  // the TMA store has read the staging box
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMiscOff + 8);
 
@@ -319,6 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(done_bar, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&stg_full[i], 128);
+            mbar_init(&stg_free[i], 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -352,11 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n0 = x.n0, n1 = x.n1;
                 if (PAGED && x.bad && x.qrow0 == 0 && x.head == 0 && elect_one() && a.err)
                     atomicOr(a.err, x.bad);
-                for (int i = 0; i < NQ && ok; ++i) {
-                    if ((i ? n1 : n0) == 0) continue;
+                auto load_q = [&](int i) {
+                    if ((i ? n1 : n0) == 0) return;
                     // the previous unit's QK^T products of this tile are done
                     if (qc[i] > 0) ok = wait_or_abort(&q_empty[i], (qc[i] - 1) & 1, a.err, abort_flag);
-                    if (!ok) break;
+                    if (!ok) return;
                     uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
                     if (elect_one()) {
                         mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
@@ -369,10 +380,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             x.head);
                         }
                     }
+                    __syncwarp();
                     ++qc[i];
-                }
+                };
+                // dense: order Q0, K0, Q1, V0, K1, ...: Q1 is released last (by
+                // the previous unit's final QK^T) and must not hold back K0,
+                // which tile 0's first QK^T of this unit needs early.  Paged K
+                // tiles take one table read and 128 / block_size copies each;
+                // there Q0, Q1, K0 measured faster.
+                load_q(0);
+                if (PAGED) load_q(1);
                 const int n_loads = 2 * max(n0, n1);
                 for (int v = 0; v < n_loads && ok; ++v, ++ukv) {
+                    if (!PAGED && v == 1) {
+                        load_q(1);
+                        if (!ok) break;
+                    }
                     const int slot = ukv % C::kStages;
                     if (ukv >= (uint32_t)C::kStages)
                         ok = wait_or_abort(&kv_empty[slot], ((ukv / C::kStages) - 1) & 1, a.err, abort_flag);
@@ -481,13 +504,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n0 = x.n0, n1 = x.n1;
                 const int nkv_max = max(n0, n1);
                 if (nkv_max == 0) continue;  // a paged unit with no rows
+                // tile 0's first QK^T goes out as soon as Q0 and K0 have landed;
+                // Q1 (released last, loaded after K0) does not hold it back
                 if (n0 > 0) ok = wait_or_abort(&q_full[0], qc0 & 1, a.err, abort_flag);
-                if (ok && n1 > 0) ok = wait_or_abort(&q_full[1], qc1 & 1, a.err, abort_flag);
                 if (ok) ok = wait_kv(ukv);
                 if (!ok) break;
                 tc_fence_after();
                 if (n0 > 0) issue_s(0, ukv);
-                if (n1 > 0) issue_s(1, ukv);
+                if (n1 > 0) {
+                    ok = wait_or_abort(&q_full[1], qc1 & 1, a.err, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(1, ukv);
+                }
                 if (elect_one()) {
                     mma_commit(&kv_empty[ukv % C::kStages]);
                     // a query tile with a single key tile has issued its only QK^T
@@ -574,7 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_tm = tmem + lane_off + i * BN;
         const uint32_t o_tm = tmem + lane_off + 2 * BN + i * 128;
         bool ok = true;
-        uint32_t itc = 0;  // key-tile iterations done by this query tile so far
+        uint32_t itc = 0;        // key-tile iterations done by this query tile so far
+        uint32_t stg_count = 0;  // O boxes staged by this warpgroup so far
         for (int rr = 0; ok; ++rr) {
             const int u = snake_unit(rr, c, G, n_units);
             if (u < 0) break;
@@ -671,21 +701,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool live = row < x.nq;
                 const size_t orow_idx = PAGED ? ((size_t)(x.qtok0 + (live ? row : 0)) * a.Hq + x.head)
                                               : ((size_t)x.head * a.N + (live ? row : 0));
-                __nv_bfloat16 *orow = a.O + orow_idx * D;
+                const int tile_row0 = x.qrow0 + i * BM;
+                if (!PAGED || tile_row0 + BM <= x.nq) {
+                    // Each thread writes its row into the tile's 128B-swizzled
+                    // staging box, 64 columns at a time, and one thread stores
+                    // the box with TMA (whole 128-byte row segments instead of
+                    // 32 rows per store instruction; rows past the end of a
+                    // dense sequence are clipped by the tensor map).
+                    const uint32_t stg = smem_base + C::kStageOff + i * kBoxBytes;
+                    const uint32_t row_addr = stg + r_in * 128;
+                    const bool issuer = quarter == 0 && lane == 0;
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t orr[32];
-                    tmem_ld32(o_tm + 32 * cc, orr);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                    for (int h = 0; h < D / 64 && ok; ++h) {
+                        uint32_t o0[32], o1[32];
+                        tmem_ld32(o_tm + 64 * h, o0);
+                        tmem_ld32(o_tm + 64 * h + 32, o1);
+                        tmem_wait_ld();
+                        uint32_t pk[32];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
-                    if (live) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cc);
+                        for (int e = 0; e < 16; ++e) {
+                            pk[e] = pack_bf16x2(__uint_as_float(o0[2 * e]) * inv, __uint_as_float(o0[2 * e + 1]) * inv);
+                            pk[16 + e] =
+                                pack_bf16x2(__uint_as_float(o1[2 * e]) * inv, __uint_as_float(o1[2 * e + 1]) * inv);
+                        }
+                        if (stg_count > 0) {
+                            ok = wait_or_abort(&stg_free[i], (stg_count - 1) & 1, a.err, abort_flag);
+                            if (!ok) break;
+                        }
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        for (int ch = 0; ch < 8; ++ch)
+                            st_shared_v4(row_addr + ((ch ^ (r_in & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
+                                         pk[4 * ch + 2], pk[4 * ch + 3]);
+                        fence_proxy_async_smem();
+                        mbar_arrive(&stg_full[i]);
+                        if (issuer) {
+                            ok = wait_or_abort(&stg_full[i], stg_count & 1, a.err, abort_flag);
+                            if (ok) {
+                                if (PAGED)
+                                    tma_store_2d(&tmO, smem + C::kStageOff + i * kBoxBytes, x.head * D + 64 * h,
+                                                 x.qtok0 + tile_row0);
+                                else
+                                    tma_store_3d(&tmO, smem + C::kStageOff + i * kBoxBytes, 64 * h, tile_row0, x.head);
+                                bulk_commit();
+                                bulk_wait_read_all();
+                                mbar_arrive(&stg_free[i]);
+                            }
+                        }
+                        ++stg_count;
+                    }
+                    if (!ok) break;
+                } else {
+                    // a paged tile that ends inside the sequence's rows: plain
+                    // stores, live rows only
+                    __nv_bfloat16 *orow = a.O + orow_idx * D;
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_tm + 32 * cc, orr);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv,
+                                                __uint_as_float(orr[2 * e + 1]) * inv);
+                        if (live) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cc);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        }
                     }
                 }
                 if (live) a.LSE[orow_idx] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
@@ -695,6 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             itc += my_nkv;
         }
+        // the staged O stores are complete before the CTA exits
+        if (quarter == 0 && lane == 0) bulk_wait_all();
         tc_fence_before();
     }
 
@@ -764,11 +850,12 @@ attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
             return ATTN_ECUDA;
         attr_set[dev] = true;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const int BH = p.B * p.H;
-    if (!make_map(&tq, p.Q, p.N, D, BH) || !make_map(&tk, p.K, p.N, D, BH) || !make_map(&tv, p.V, p.N, D, BH))
+    if (!make_map(&tq, p.Q, p.N, D, BH) || !make_map(&tk, p.K, p.N, D, BH) || !make_map(&tv, p.V, p.N, D, BH) ||
+        !make_map(&to, p.O, p.N, D, BH))
         return ATTN_ECUDA;
-    PrefillArgs a;
+    PrefillArgs a = {};
     a.O = static_cast<__nv_bfloat16 *>(p.O);
     a.LSE = p.LSE;
     a.err = p.err_flag;
@@ -784,7 +871,7 @@ attn_status launch_t(const DenseLaunch &p, cudaStream_t stream) {
     // each walking its units in snake order
     const long long units = (long long)a.nblk * BH;
     const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
-    prefill_bf16_kernel<D, CAUSAL, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+    prefill_bf16_kernel<D, CAUSAL, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
@@ -804,11 +891,12 @@ attn_status launch_paged_t(const PagedPrefillLaunch &p, cudaStream_t stream) {
     if (sm_count[dev] == 0 &&
         cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return ATTN_ECUDA;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const long long cache_rows = (long long)p.num_blocks * p.Hkv * p.block_size;
     if (!make_map_2d(&tq, p.q, (long long)p.Hq * D, p.total_q, (long long)p.Hq * D, BM) ||
         !make_map_2d(&tk, p.k_cache, D, cache_rows, D, p.block_size) ||
-        !make_map_2d(&tv, p.v_cache, D, cache_rows, D, p.block_size))
+        !make_map_2d(&tv, p.v_cache, D, cache_rows, D, p.block_size) ||
+        !make_map_2d(&to, p.O, (long long)p.Hq * D, p.total_q, (long long)p.Hq * D, BM))
         return ATTN_ECUDA;
     PrefillArgs a = {};
     a.O = static_cast<__nv_bfloat16 *>(p.O);
@@ -829,7 +917,7 @@ attn_status launch_paged_t(const PagedPrefillLaunch &p, cudaStream_t stream) {
     const long long units = (long long)a.nqb * a.S * a.Hq;
     if (units == 0) return ATTN_OK;
     const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
-    prefill_bf16_kernel<D, true, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+    prefill_bf16_kernel<D, true, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
