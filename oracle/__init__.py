@@ -24,3 +24,4 @@ from .attention import (  # noqa: F401
     softmax_probs,
 )
 from .brute import brute_attention, brute_paged_decode, build_brute  # noqa: F401
+from . import fp8  # noqa: F401,E402  (e4m3 block quantisation with incoherent processing)
