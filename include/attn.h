@@ -162,6 +162,44 @@ ATTN_API attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, c
                                            attn_stream_t stream);
 
 /*
+ * FP8 prefill, step 1: block quantisation of Q or K to e4m3
+ * ("一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解" §二
+ * "FlashAttention-3改进": the GEMMs run on FP8 tensor cores; block
+ * quantisation and incoherent processing limit the accuracy lost).
+ *
+ * x      : bf16 [BH, N, d] (device), d = 128.
+ * codes  : e4m3 [BH, N, d] (device, one byte per element, caller-owned).
+ * scales : fp32 [BH, ceil(N / 128)] (device): one dequantisation scale per
+ *          block of 128 rows of one head.
+ * signs  : null, or d int8 values of +1 / -1 (device): incoherent processing,
+ *          each row is multiplied by diag(signs) and the Sylvester Hadamard
+ *          matrix before quantisation.  Give Q and K the same signs: the
+ *          1/sqrt(d) of the rotation is folded into the scales, so the
+ *          dequantised operands keep Q K^T.
+ * Per block: amax = max |y| (y the rotated or plain rows, fp32);
+ * code = e4m3(y * fp32(448 / amax)) rounded to nearest even, saturating;
+ * scale = amax / 448 (/ sqrt(d) with rotation); an all-zero block has
+ * scale 1 and zero codes.
+ * Errors: ATTN_EUNSUPPORTED for d != 128; ATTN_EINVAL for null or unaligned
+ * pointers (x, codes 16-byte; scales 4-byte).  BH = 0 or N = 0: no-op.
+ */
+ATTN_API attn_status attn_quantize_fp8(const void *x, void *codes, float *scales, int BH, int N, int d,
+                                       const int8_t *signs, attn_stream_t stream);
+
+/*
+ * FP8 prefill, step 2: attn_fwd with e4m3 Q and K (from attn_quantize_fp8)
+ * and bf16 V.  S = (Q8 * q_scale)(K8 * k_scale)^T is computed on tcgen05
+ * tensor cores (kind::f8f6f4, fp32 accumulation); the per-block scales
+ * fold into the softmax scale, so the online softmax, P.V (bf16) and the
+ * outputs are those of attn_fwd.  O bf16 [B, H, N, d], LSE fp32 [B, H, N];
+ * d = 128; causal as attn_fwd.
+ * Errors: as attn_fwd (q8, k8, V, O 16-byte aligned; scales and LSE 4-byte).
+ */
+ATTN_API attn_status attn_fwd_fp8(const void *q8, const float *q_scale, const void *k8, const float *k_scale,
+                                  const void *V, void *O, float *LSE, int B, int H, int N, int d, int causal,
+                                  float scale, int32_t *err_flag, attn_stream_t stream);
+
+/*
  * Multi-token paged prefill (chunked prefill / prefix reuse): several new
  * query tokens per sequence attend causally to that sequence's paged cache,
  * which already holds their own keys and values ("第 2 章核心模块：

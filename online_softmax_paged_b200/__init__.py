@@ -18,6 +18,7 @@ __all__ = [
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
     "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
+    "attn_quantize_fp8", "attn_fwd_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +31,7 @@ ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_I
 # every function include/attn.h declares
 EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
                     "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_attn_prefill",
+                    "attn_quantize_fp8", "attn_fwd_fp8",
                     "paged_kv_append",
                     "paged_block_copy",
                     "attn_read_error", "attn_status_str")
@@ -75,6 +77,10 @@ def load():
     lib.paged_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                               c_float, c_int, vp, vp]
     lib.paged_attn_decode_noalloc.restype = c_int
+    lib.attn_quantize_fp8.argtypes = [vp, vp, vp, c_int, c_int, c_int, vp, vp]
+    lib.attn_quantize_fp8.restype = c_int
+    lib.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_float, vp, vp]
+    lib.attn_fwd_fp8.restype = c_int
     lib.paged_attn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
                                        c_int, c_int, c_int, c_float, c_int, vp, vp]
     lib.paged_attn_prefill.restype = c_int
@@ -139,6 +145,60 @@ def attn_fwd(Q, K, V, O=None, LSE=None, causal=False, scale=None, err_flag=None,
                          float(scale), _dtype_code(Q.dtype), _ptr(err_flag), _stream(stream, Q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return O, LSE
+
+
+def attn_quantize_fp8(x, signs=None, codes=None, scales=None, stream=None):
+    """Block-quantise bf16 rows x [..., N, d] (d = 128, contiguous) to e4m3
+    with one scale per 128 rows of each leading index; ``signs`` (d int8
+    values of +-1) turns on incoherent processing.  Returns (codes uint8,
+    same shape as x, viewable as torch.float8_e4m3fn; scales fp32
+    [..., ceil(N / 128)]).  See include/attn.h."""
+    _check_cuda(x, signs, codes, scales)
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be contiguous bf16")
+    *lead, N, d = x.shape
+    BH = int(math.prod(lead)) if lead else 1
+    nblk = -(-N // 128)
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(tuple(lead) + (nblk,), dtype=torch.float32, device=x.device)
+    if signs is not None and (signs.dtype != torch.int8 or signs.numel() != d):
+        raise ValueError("signs must be d int8 values")
+    st = load().attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(scales), BH, N, d, _ptr(signs), _stream(stream, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_quantize_fp8")
+    return codes, scales
+
+
+def attn_fwd_fp8(q8, q_scale, k8, k_scale, V, O=None, LSE=None, causal=False, scale=None, err_flag=None,
+                 stream=None):
+    """FP8 prefill: e4m3 Q and K [B, H, N, d] (uint8 or float8_e4m3fn) with
+    their block scales [B, H, ceil(N / 128)] from attn_quantize_fp8, bf16 V
+    [B, H, N, d].  Returns (O bf16, LSE fp32).  See include/attn.h."""
+    _check_cuda(q8, q_scale, k8, k_scale, V, O, LSE, err_flag)
+    B, H, N, d = V.shape
+    if q8.shape != V.shape or k8.shape != V.shape or q8.element_size() != 1 or k8.element_size() != 1:
+        raise ValueError("q8 and k8 must be one-byte tensors of V's shape")
+    if V.dtype != torch.bfloat16:
+        raise ValueError("V must be bf16")
+    for t in (q8, q_scale, k8, k_scale, V):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    nblk = -(-N // 128)
+    if q_scale.shape != (B, H, nblk) or k_scale.shape != (B, H, nblk):
+        raise ValueError("scales must be [B, H, ceil(N / 128)]")
+    if O is None:
+        O = torch.empty_like(V)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=V.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = load().attn_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(V), _ptr(O), _ptr(LSE), B, H,
+                             N, d, int(bool(causal)), float(scale), _ptr(err_flag), _stream(stream, V.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
     return O, LSE
 
 

@@ -32,6 +32,32 @@ attn_status attn_fwd(const void *Q, const void *K, const void *V, void *O, float
     return dt == ATTN_BF16 ? osp::launch_prefill_bf16(p, s) : osp::launch_dense_f32(p, s);
 }
 
+attn_status attn_quantize_fp8(const void *x, void *codes, float *scales, int BH, int N, int d, const int8_t *signs,
+                              attn_stream_t stream) {
+    if (BH < 0 || N < 0) return ATTN_EINVAL;
+    if (d != 128) return ATTN_EUNSUPPORTED;
+    if (BH == 0 || N == 0) return ATTN_OK;
+    if (!x || !codes || !scales) return ATTN_EINVAL;
+    if (!aligned16(x) || !aligned16(codes) || ((uintptr_t)scales & 3u)) return ATTN_EINVAL;
+    osp::QuantLaunch p{x, codes, scales, signs, BH, N};
+    return osp::launch_quantize_fp8(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_fwd_fp8(const void *q8, const float *q_scale, const void *k8, const float *k_scale, const void *V,
+                         void *O, float *LSE, int B, int H, int N, int d, int causal, float scale, int32_t *err_flag,
+                         attn_stream_t stream) {
+    if (!q8 || !q_scale || !k8 || !k_scale || !V || !O || !LSE) return ATTN_EINVAL;
+    if (B < 1 || H < 1 || N < 1) return ATTN_EINVAL;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
+    if (d != 128) return ATTN_EUNSUPPORTED;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(V) || !aligned16(O) || ((uintptr_t)LSE & 3u) ||
+        ((uintptr_t)q_scale & 3u) || ((uintptr_t)k_scale & 3u))
+        return ATTN_EINVAL;
+    if ((long long)B * H > 0x7fffffffLL / 2) return ATTN_EINVAL;
+    osp::Fp8Launch p{q8, k8, V, q_scale, k_scale, O, LSE, B, H, N, causal ? 1 : 0, scale, err_flag};
+    return osp::launch_prefill_fp8(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq, int block_size) {
     if (num_seqs < 0 || H < 1 || d != 128 || max_blocks_per_seq < 1 || block_size < 16 || block_size % 16)
         return 0;

@@ -57,7 +57,27 @@ struct PagedPrefillLaunch {
     int32_t *err_flag;
 };
 
+struct QuantLaunch {
+    const void *x;        // bf16 [BH, N, d]
+    void *codes;          // e4m3 [BH, N, d]
+    float *scales;        // [BH, ceil(N / 128)]
+    const int8_t *signs;  // d entries of +-1, or null (no rotation)
+    int BH, N;
+};
+
+struct Fp8Launch {
+    const void *q8, *k8, *V;
+    const float *q_scale, *k_scale;
+    void *O;
+    float *LSE;
+    int B, H, N, causal;
+    float scale;
+    int32_t *err_flag;
+};
+
 attn_status launch_dense_f32(const DenseLaunch &p, cudaStream_t stream);
+attn_status launch_quantize_fp8(const QuantLaunch &p, cudaStream_t stream);
+attn_status launch_prefill_fp8(const Fp8Launch &p, cudaStream_t stream);
 attn_status launch_paged_prefill(const PagedPrefillLaunch &p, cudaStream_t stream);
 attn_status launch_kv_append(const AppendLaunch &p, cudaStream_t stream);
 attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream);

@@ -86,6 +86,10 @@ struct PrefillArgs {
     // q / O / LSE, at key positions seq_lens[s] - n_s .. seq_lens[s] - 1
     const int32_t *cu_q, *seq_lens, *block_table;
     int S, Hq, Hkv, max_blocks, num_blocks, block_size, nqb, total_q;
+    // FP8 mode: e4m3 Q and K with one dequantisation scale per 128-row block
+    // ([B*H, nsblk] each); V stays bf16
+    const float *q_scale, *k_scale;
+    int nsblk;
 };
 
 // What every role needs to know about a work unit (256 query rows of one
@@ -106,6 +110,15 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
     d |= (uint64_t)1 << 46;  // descriptor version for sm_100
     d |= (uint64_t)2 << 61;  // 128-byte swizzle
     return d;
+}
+
+// kind::f8f6f4 instruction descriptor: e4m3 A and B, both K-major, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4)                           // D: fp32
+           | (0u << 7)                         // A: e4m3
+           | (0u << 10)                        // B: e4m3
+           | ((uint32_t)(N >> 3) << 17)        // N / 8
+           | ((uint32_t)(M >> 4) << 24);       // M / 16
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
@@ -287,12 +300,16 @@ __device__ __forceinline__ void get_unit(const PrefillArgs &a, bool causal, int 
     x.n1 = n[1];
 }
 
-template <int D, bool CAUSAL, bool PAGED>
+template <int D, bool CAUSAL, bool PAGED, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                         PrefillArgs a) {
     using C = Cfg<D>;
+    static_assert(!F8 || (D == 128 && !PAGED), "FP8 QK^T: dense, d = 128");
+    // Q and K tiles: bf16 in 64-column boxes, or e4m3 in one 128-byte-wide box
+    constexpr int kQKBytes = F8 ? BM * D : C::kTileBytes;
+    constexpr int kQKBoxes = F8 ? 1 : C::kBoxes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -370,8 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) return;
                     uint8_t *dst = smem + C::kQOff + i * C::kTileBytes;
                     if (elect_one()) {
-                        mbar_arrive_expect_tx(&q_full[i], C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b) {
+                        mbar_arrive_expect_tx(&q_full[i], kQKBytes);
+                        for (int b = 0; b < kQKBoxes; ++b) {
                             if (PAGED)  // rows past the sequence's tokens are loaded but never stored
                                 tma_load_2d(dst + b * kBoxBytes, &tmQ, &q_full[i], x.head * D + b * kBoxCols,
                                             x.qtok0 + x.qrow0 + i * BM);
@@ -403,9 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const CUtensorMap *tm = (v & 1) ? &tmV : &tmK;
                     uint8_t *dst = smem + C::kRingOff + slot * C::kTileBytes;
                     if (!PAGED) {
+                        const bool qk = F8 && !(v & 1);  // an e4m3 K tile
                         if (elect_one()) {
-                            mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
-                            for (int b = 0; b < C::kBoxes; ++b)
+                            mbar_arrive_expect_tx(&kv_full[slot], qk ? kQKBytes : C::kTileBytes);
+                            for (int b = 0; b < (qk ? kQKBoxes : C::kBoxes); ++b)
                                 tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN,
                                             x.head);
                         }
@@ -453,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
+            constexpr uint32_t idesc_qk8 = idesc_e4m3_f32(BM, BN);
             // base descriptors; per-slot and per-k-step offsets are added to the
             // start-address field (16-byte units, no carry: smem < 256 KiB)
             const uint64_t dq0 = desc_sw128(smem_base + C::kQOff, 16, 1024);
@@ -472,10 +491,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t da = i ? dq1 : dq0, db = dk + slot_off(u);
                 const uint32_t d_tm = i ? tm_s1 : tm_s0;
                 if (elect_one()) {
+                    if constexpr (F8) {
+                        // e4m3 rows are 128 bytes: K = 32 per instruction, 32 bytes apart
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint64_t off = (uint64_t)(((ks / 4) * kBoxBytes + (ks % 4) * 32) >> 4);
-                        mma_ss(d_tm, da + off, db + off, idesc_qk, ks > 0);
+                        for (int ks = 0; ks < D / 32; ++ks) {
+                            const uint64_t off = (uint64_t)((ks * 32) >> 4);
+                            mma_ss_f8(d_tm, da + off, db + off, idesc_qk8, ks > 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint64_t off = (uint64_t)(((ks / 4) * kBoxBytes + (ks % 4) * 32) >> 4);
+                            mma_ss(d_tm, da + off, db + off, idesc_qk, ks > 0);
+                        }
                     }
                     mma_commit(&s_full[i]);
                 }
@@ -613,6 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int my_nkv = i ? x.n1 : x.n0;
             const int tile_pos = x.pos0 + x.qrow0 + i * BM;  // key position of the tile's row 0
             const int row = x.qrow0 + i * BM + r_in;        // query row in the sequence
+            // FP8: the dequantisation scales of this query tile and of each key
+            // tile fold into the softmax scale
+            const float c_unit =
+                (F8 && my_nkv > 0) ? a.scale_log2 * __ldg(a.q_scale + (size_t)x.head * a.nsblk + (x.qrow0 + i * BM) / BM)
+                                   : a.scale_log2;
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < my_nkv; ++j) {
                 ok = wait_or_abort(&s_full[i], (itc + j) & 1, a.err, abort_flag);
@@ -651,12 +684,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 const float mx =
                     max3(max3(mxa[0], mxa[1], mxa[2]), max3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
-                const float mx2 = mx * a.scale_log2;
+                const float c_step = F8 ? c_unit * __ldg(a.k_scale + (size_t)x.head * a.nsblk + j) : c_unit;
+                const float mx2 = mx * c_step;
                 float m_ref = m;
                 if (mx2 > m + kRescaleThreshold) m_ref = mx2;
                 if (m_ref == -INFINITY) m_ref = 0.f;  // row with nothing visible yet
                 const float alpha = ex2_approx(m - m_ref);
-                const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
+                const uint64_t scale2 = f2_pack(c_step, c_step);
                 const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
                 uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
                 if (masked)
@@ -921,7 +955,64 @@ attn_status launch_paged_t(const PagedPrefillLaunch &p, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
+// [B*H, N, d] e4m3 (bytes) viewed as a 3-D tensor map, box 128 x 128 x 1
+// (one 128-byte row per box row), 128B swizzle.
+bool make_map_u8(CUtensorMap *m, const void *base, int N, int d, int BH) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)N * d};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool CAUSAL>
+attn_status launch_fp8_t(const Fp8Launch &p, cudaStream_t stream) {
+    constexpr int D = 128;
+    using C = Cfg<D>;
+    static bool attr_set[64] = {false};
+    static int sm_count[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ECUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(prefill_bf16_kernel<D, CAUSAL, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+            return ATTN_ECUDA;
+        attr_set[dev] = true;
+    }
+    if (sm_count[dev] == 0 &&
+        cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ECUDA;
+    const int BH = p.B * p.H;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_map_u8(&tq, p.q8, p.N, D, BH) || !make_map_u8(&tk, p.k8, p.N, D, BH) ||
+        !make_map(&tv, p.V, p.N, D, BH) || !make_map(&to, p.O, p.N, D, BH))
+        return ATTN_ECUDA;
+    PrefillArgs a = {};
+    a.O = static_cast<__nv_bfloat16 *>(p.O);
+    a.LSE = p.LSE;
+    a.err = p.err_flag;
+    a.N = p.N;
+    a.BH = BH;
+    a.nblk = (p.N + NQ * BM - 1) / (NQ * BM);
+    a.scale_log2 = p.scale * 1.4426950408889634f;
+    a.q_scale = p.q_scale;
+    a.k_scale = p.k_scale;
+    a.nsblk = (p.N + BM - 1) / BM;
+    const long long units = (long long)a.nblk * BH;
+    const int grid = (int)(units < sm_count[dev] ? units : sm_count[dev]);
+    prefill_bf16_kernel<D, CAUSAL, false, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
 }  // namespace
+
+attn_status launch_prefill_fp8(const Fp8Launch &p, cudaStream_t stream) {
+    return p.causal ? launch_fp8_t<true>(p, stream) : launch_fp8_t<false>(p, stream);
+}
 
 attn_status launch_paged_prefill(const PagedPrefillLaunch &p, cudaStream_t stream) {
     return p.d == 128 ? launch_paged_t<128>(p, stream) : launch_paged_t<64>(p, stream);

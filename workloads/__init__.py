@@ -267,6 +267,14 @@ def paged_chunked_prefill(num_seqs=8, Hq=32, Hkv=8, d=128, block_size=16, pool=2
     return paged_prefill_inputs(ctx, [chunk] * num_seqs, Hq, Hkv, d, block_size, pool, seed, device, dtype, mb)
 
 
+def hadamard_signs(d=128, seed=0, device="cpu") -> torch.Tensor:
+    """The random diagonal of incoherent processing: d int8 values, each +1
+    or -1 with probability 1/2 (torch.randint from a CPU generator seeded
+    ``seed``)."""
+    g = _gen(seed, "cpu")
+    return (torch.randint(0, 2, (d,), generator=g, dtype=torch.int8) * 2 - 1).to(device)
+
+
 def shuffle_placement(inp: PagedInputs, seed=1, pool=None) -> PagedInputs:
     """Same logical data, new physical placement: every used physical block is
     moved to a new id by a random permutation of the pool, and the table is
