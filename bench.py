@@ -12,6 +12,8 @@ A step is one call of the entry point on one batch of the workload:
   decode_gqa_g4/_g8    paged_attn_decode_gqa, decode_uniform with 32 query heads over 8 / 4 K/V heads
   kv_append            paged_kv_append, 64 seqs x 512 new tokens (H=32, d=128, bs=16)
   block_copy           paged_block_copy, 1024 block pairs (copy-on-write), 128 KiB per block
+  prefill_fp8_2k / _16k the prefill workloads through the FP8 path: attn_quantize_fp8 of Q and K
+                       (incoherent processing on) + attn_fwd_fp8 (e4m3 QK^T, bf16 P.V)
   prefill_paged_chunked paged_attn_prefill, 8 seqs x 2048 new tokens after U{0..6144} cached,
                        32 query heads over 8 K/V heads, d=128, bs=16
 The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
@@ -522,6 +524,114 @@ class BlockCopy:
         return self.work * n / self.cfg["pairs"], dt, f"{n} of {self.cfg['pairs']} pairs"
 
 
+class Fp8Prefill:
+    """The causal prefill workloads through the FP8 path: one step =
+    attn_quantize_fp8(Q), attn_quantize_fp8(K) (random-sign Hadamard
+    incoherent processing), attn_fwd_fp8.  Work = the bf16 prefill's FLOPs.
+    The roofline is that of the attention kernel alone, timed with its own
+    events; its peak blends the two contractions: QK^T at the e4m3 rate
+    (2x bf16, the nominal ratio) and P.V at the bf16 rate, i.e. a time at
+    peak of 0.75 x that of an all-bf16 kernel."""
+
+    def __init__(self, cfg, name, device, seed=0):
+        self.name = name
+        self.cfg = cfg
+        self.B, self.H, self.N, self.d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+        one = 3 * self.B * self.H * self.N * self.d * 2
+        self.copies = max(1, math.ceil(3 * L2_BYTES / one))
+        self.sets = [W.dense_inputs(self.B, self.H, self.N, self.d, dtype=cfg["dtype"], mult=cfg["mult"],
+                                    seed=seed + i, device=device, causal=True) for i in range(self.copies)]
+        self.signs = W.hadamard_signs(self.d, seed=seed, device=device)
+        nblk = -(-self.N // 128)
+        shp = (self.B, self.H, self.N, self.d)
+        self.q8 = torch.empty(shp, dtype=torch.uint8, device=device)
+        self.k8 = torch.empty(shp, dtype=torch.uint8, device=device)
+        self.qs = torch.empty((self.B, self.H, nblk), dtype=torch.float32, device=device)
+        self.ks = torch.empty((self.B, self.H, nblk), dtype=torch.float32, device=device)
+        self.O = torch.empty(shp, dtype=torch.bfloat16, device=device)
+        self.LSE = torch.empty((self.B, self.H, self.N), dtype=torch.float32, device=device)
+        self.work = 4.0 * self.B * self.H * self.d * (self.N * (self.N + 1) // 2)
+        self.unit, self.scale_unit = "TFLOP/s", 1e12
+        self.launches_per_step = 3
+        self.kernel = "prefill_bf16_kernel"
+        self.peak_factor = 1.0 / 0.75
+        self.kernel_events = []
+        self.record = False
+
+    def step(self, i, osp):
+        s = self.sets[i % self.copies]
+        osp.attn_quantize_fp8(s["Q"], signs=self.signs, codes=self.q8, scales=self.qs)
+        osp.attn_quantize_fp8(s["K"], signs=self.signs, codes=self.k8, scales=self.ks)
+        if self.record:
+            st = torch.cuda.current_stream()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+        osp.attn_fwd_fp8(self.q8, self.qs, self.k8, self.ks, s["V"], O=self.O, LSE=self.LSE, causal=True,
+                         scale=s["scale"])
+        if self.record:
+            e1.record(st)
+            self.kernel_events.append((e0, e1))
+
+    def config(self):
+        return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N, "d": self.d, "causal": True,
+                "dtype": "e4m3 Q/K, bf16 V/P/O", "global_batch": self.B, "seq_len": self.N,
+                "incoherent_processing": True,
+                "l2": f"inputs rotate over {self.copies} copies "
+                      f"({self.copies * 3 * self.B * self.H * self.N * self.d * 2 / 2**20:.0f} MiB > L2)"}
+
+    def e2e(self, osp, steps, device):
+        s = self.sets[0]
+        hq, hk, hv = (s[k].cpu().pin_memory() for k in ("Q", "K", "V"))
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty(self.LSE.shape, dtype=torch.float32).pin_memory()
+        dq, dk, dv = torch.empty_like(s["Q"]), torch.empty_like(s["K"]), torch.empty_like(s["V"])
+        st = torch.cuda.current_stream(device)
+
+        def one():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            osp.attn_quantize_fp8(dq, signs=self.signs, codes=self.q8, scales=self.qs)
+            osp.attn_quantize_fp8(dk, signs=self.signs, codes=self.k8, scales=self.ks)
+            osp.attn_fwd_fp8(self.q8, self.qs, self.k8, self.ks, dv, O=self.O, LSE=self.LSE, causal=True,
+                             scale=s["scale"])
+            ho.copy_(self.O, non_blocking=True)
+            hl.copy_(self.LSE, non_blocking=True)
+
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / steps
+        return ms, 3 * hq.numel() * 2, ho.numel() * 2 + hl.numel() * 4
+
+    def cpu_sample(self, budget_s):
+        """The oracle's quantisation of one (b, h) head's Q and K and exact
+        attention on the dequantised operands, head after head, until the budget."""
+        import numpy as np
+        import oracle
+        from oracle import fp8 as F
+        s = self.sets[0]
+        sg = self.signs.cpu().numpy()
+        done, t0 = 0, time.perf_counter()
+        heads = [(b, h) for b in range(self.B) for h in range(self.H)]
+        for b, h in heads:
+            q = F.dequantize_blocks(*F.quantize_blocks(s["Q"][b, h].float().cpu().numpy()[None], 128, signs=sg))[0]
+            k = F.dequantize_blocks(*F.quantize_blocks(s["K"][b, h].float().cpu().numpy()[None], 128, signs=sg))[0]
+            v = s["V"][b, h].float().cpu().numpy().astype(np.float64)
+            oracle.attention_head(q, k, v, True, s["scale"])
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return self.work * done / len(heads), dt, f"{done} of {len(heads)} (b, h) heads of {self.name}, full rows"
+
+
 class PagedPrefill:
     """paged_attn_prefill on the chunked-prefill workload.  Work = 4 * d *
     H_q * (visible query-key pairs), new token i of sequence s seeing
@@ -649,6 +759,10 @@ def make_workload(name, device, seed=0):
         return BlockCopy(name, device, seed)
     if name == "prefill_paged_chunked":
         return PagedPrefill(name, device, seed)
+    if name == "prefill_fp8_2k":
+        return Fp8Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
+    if name == "prefill_fp8_16k":
+        return Fp8Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -675,6 +789,9 @@ def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0):
     t_region0 = time.perf_counter()
     g0 = torch.cuda.Event(enable_timing=True)
     g1 = torch.cuda.Event(enable_timing=True)
+    if hasattr(wl, "kernel_events"):  # steps of several launches time the dominant one too
+        wl.kernel_events.clear()
+        wl.record = True
     g0.record(st)
     for i in range(steps):
         evs[i][0].record(st)
@@ -685,6 +802,9 @@ def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0):
     barrier(ws)
     wall = time.perf_counter() - t_region0
     per = [a.elapsed_time(b) for a, b in evs]
+    if hasattr(wl, "kernel_events"):
+        wl.record = False
+        per = [a.elapsed_time(b) for a, b in wl.kernel_events]
     total_ms = g0.elapsed_time(g1)
     return per, total_ms, wall
 
@@ -703,9 +823,13 @@ def roofline(wl, per_ms, pk, pk_src, bound, clocks=None):
         capped = bool(clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
                       and "sw_power_cap" in clocks.get("reasons", [])
                       and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+        f = getattr(wl, "peak_factor", 1.0)  # FP8 QK^T: the blended e4m3 / bf16 peak
+        burst, sustained = burst * f, sustained * f
         peak = sustained if capped else burst
         extra = {"peak_kind": "sustained (power-capped clocks in the timed window)" if capped else "burst",
                  "frac_of_burst": round(achieved / burst, 4), "frac_of_sustained": round(achieved / sustained, 4)}
+        if f != 1.0:
+            extra["peak_kind"] += "; bf16 peak x 4/3 (QK^T at the e4m3 rate, P.V at the bf16 rate)"
         unit = "TFLOP/s"
     else:
         peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -730,7 +854,7 @@ def run_ours(args):
     pk, pk_src = peaks()
 
     wl = make_workload(args.workload, device, seed=args.seed + rank)
-    bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill)) else "hbm"
+    bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill, Fp8Prefill)) else "hbm"
     with ClockSampler(local) as clocks:
         t_load0 = time.perf_counter()
         per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak)
@@ -766,7 +890,8 @@ def run_ours(args):
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16)",
+                "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16" if isinstance(wl, Fp8Prefill) else "bf16",
+                "data": "synthetic (seeded N(0,1), bf16)",
                 "config": {**wl.config(), "parallelism": f"replicas{ws}" if ws > 1 else "single"},
                 "roofline": rl, "cpu_baseline": cpu,
                 "e2e": {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d,
@@ -812,6 +937,27 @@ def run_reference(args):
 
         sample = f"16 new-token rows of one (sequence, head) of {name} per step"
         config = wl.config()
+    elif name.startswith("prefill_fp8"):
+        from oracle import fp8 as F
+        cfg = W.PREFILL_CAUSAL_2K if name.endswith("2k") else W.PREFILL_CAUSAL_16K
+        B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+        per_head = 4.0 * d * (N * (N + 1) // 2)
+        unit, su = "TFLOP/s", 1e12
+        inp = W.dense_inputs(B, H, N, d, dtype=cfg["dtype"], mult=cfg["mult"], seed=args.seed, device=dev,
+                             causal=True)
+        sg = W.hadamard_signs(d, seed=args.seed).numpy()
+        heads = [(b, h) for b in range(B) for h in range(H)]
+
+        def one(i):
+            b, h = heads[i % len(heads)]
+            q = F.dequantize_blocks(*F.quantize_blocks(inp["Q"][b, h].float().cpu().numpy()[None], 128, signs=sg))[0]
+            k = F.dequantize_blocks(*F.quantize_blocks(inp["K"][b, h].float().cpu().numpy()[None], 128, signs=sg))[0]
+            oracle.attention_head(q, k, inp["V"][b, h].float().cpu().numpy().astype(np.float64), True, inp["scale"])
+            return per_head
+
+        sample = f"one (b, h) head of {name} per step (quantise Q, K; exact attention)"
+        config = {"workload": name, "B": B, "H": H, "N": N, "d": d, "causal": True,
+                  "dtype": "e4m3 Q/K, bf16 V/P/O", "global_batch": B, "seq_len": N}
     elif name.startswith("prefill"):
         cfg = W.PREFILL_CAUSAL_2K if name == "prefill_2k" else W.PREFILL_CAUSAL_16K
         B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
@@ -882,7 +1028,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="prefill_2k",
                     choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
                              "decode_uniform_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8",
-                             "prefill_paged_chunked"])
+                             "prefill_paged_chunked", "prefill_fp8_2k", "prefill_fp8_16k"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")

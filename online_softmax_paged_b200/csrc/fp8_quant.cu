@@ -18,7 +18,9 @@
 // x), and (Q D H)(K D H)^T / d = Q K^T keeps the attention scores.
 // The bf16 block is read with coalesced 16-byte loads into a swizzled shared
 // buffer (chunk c of row r at c ^ (r & 15): conflict-free row reads), and the
-// codes leave the same way.  HBM-bound: 2 bytes in, 1 byte out per element.
+// codes leave the same way.  The random signs are applied as XOR masks on the
+// bf16 bits (kept in shared memory) and the butterflies of stride >= 2 run on
+// packed fp32 pairs.  HBM-bound: 2 bytes in, 1 byte out per element.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -40,6 +42,7 @@ __global__ void __launch_bounds__(kQRows) quantize_qk_kernel(const __nv_bfloat16
     constexpr int kChunks = D / 8;  // 16-byte chunks of a bf16 row
     __shared__ __align__(16) uint8_t buf[kQRows * D * 2];
     __shared__ float warp_max[kQRows / 32];
+    __shared__ __align__(16) uint32_t sign_mask[D / 2];  // per bf16x2 word: the sign bits to flip
     const int t = threadIdx.x;
     const int bh = blockIdx.x / nblk, b = blockIdx.x - bh * nblk;
     const int r0 = b * kQRows;
@@ -47,6 +50,8 @@ __global__ void __launch_bounds__(kQRows) quantize_qk_kernel(const __nv_bfloat16
     const size_t base = ((size_t)bh * N + r0) * D;
 
     // coalesced load of the block (rows * D bf16, contiguous)
+    if (ROT && t < D / 2)
+        sign_mask[t] = (__ldg(signs + 2 * t) < 0 ? 0x8000u : 0u) | (__ldg(signs + 2 * t + 1) < 0 ? 0x80000000u : 0u);
     const uint4 *src = reinterpret_cast<const uint4 *>(x + base);
     for (int k = t; k < rows * kChunks; k += kQRows) {
         const int r = k / kChunks, c = k - r * kChunks;
@@ -59,7 +64,14 @@ __global__ void __launch_bounds__(kQRows) quantize_qk_kernel(const __nv_bfloat16
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
             const uint4 w = *reinterpret_cast<const uint4 *>(buf + t * D * 2 + ((c ^ (t & (kChunks - 1))) << 4));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            if (ROT) {
+                const uint4 mk = *reinterpret_cast<const uint4 *>(sign_mask + 4 * c);
+                ws[0] ^= mk.x;
+                ws[1] ^= mk.y;
+                ws[2] ^= mk.z;
+                ws[3] ^= mk.w;
+            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 v[8 * c + 2 * e] = bf16lo(ws[e]);
@@ -71,18 +83,22 @@ __global__ void __launch_bounds__(kQRows) quantize_qk_kernel(const __nv_bfloat16
         for (int k = 0; k < D; ++k) v[k] = 0.f;
     }
     if (ROT) {
+        // y = v H: butterflies of stride 1 (scalar), then 2, ..., D/2 on
+        // packed pairs (each lane rounds as a scalar would)
 #pragma unroll
-        for (int k = 0; k < D; ++k)
-            if (__ldg(signs + k) < 0) v[k] = -v[k];
-        // y = v H: butterflies of stride 1, 2, ..., D/2 (Sylvester order)
+        for (int k = 0; k < D; k += 2) {
+            const float p = v[k], q = v[k + 1];
+            v[k] = __fadd_rn(p, q);
+            v[k + 1] = __fsub_rn(p, q);
+        }
 #pragma unroll
-        for (int h = 1; h < D; h <<= 1)
+        for (int h = 2; h < D; h <<= 1)
 #pragma unroll
-            for (int k = 0; k < D; ++k)
+            for (int k = 0; k < D; k += 2)
                 if ((k & h) == 0) {
-                    const float p = v[k], q = v[k + h];
-                    v[k] = __fadd_rn(p, q);
-                    v[k + h] = __fsub_rn(p, q);
+                    const uint64_t p = f2_pack(v[k], v[k + 1]), q = f2_pack(v[k + h], v[k + h + 1]);
+                    f2_unpack(f2_add(p, q), v[k], v[k + 1]);
+                    f2_unpack(f2_sub(p, q), v[k + h], v[k + h + 1]);
                 }
     }
     float amax = 0.f;
