@@ -256,6 +256,8 @@ __device__ __forceinline__ void final_store(const DecodeArgs &a, size_t sh, int 
     if (lane == 0) a.LSE[sh] = lse;
 }
 
+__device__ __forceinline__ void merge_row(const DecodeArgs &a, int s, size_t sh, int nsplit, int lane);
+
 // Output of a finished item: the final row for a one-split sequence, else a
 // partial; the warp completing the last split of (s, h) merges in split order.
 __device__ __forceinline__ void finish_item(const DecodeArgs &a, int s, int hq, int p, int lane, float m, float l,
@@ -267,6 +269,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, int s, int hq, 
     const int nsplit = a.item_start[s + 1] - a.item_start[s];  // (L2-resident, once per item)
     const size_t sh = (size_t)s * a.H + hq;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    (void)half;
     if (nsplit == 1) {
         if (saw_bad)
             final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
@@ -291,15 +294,24 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, int s, int hq, 
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
     __threadfence();
+    merge_row(a, s, sh, nsplit, lane);
+}
+
+// The final row of (sequence s, query head) sh from its nsplit normalised
+// partials, in split order (all lanes; lane l owns dims 4l .. 4l+3).
+__device__ __forceinline__ void merge_row(const DecodeArgs &a, int s, size_t sh, int nsplit, int lane) {
     if (__ldcg(a.seq_bad + s)) {
-        final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
+        *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = make_uint2(0u, 0u);
+        if (lane == 0) a.LSE[sh] = -INFINITY;
         return;
     }
     const float *plse = a.part_lse + sh * a.max_splits;
     float M = -INFINITY;
+#pragma unroll 4
     for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(plse + q));
     float tot = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int q = 0; q < nsplit; ++q) {
         const float w = ex2_approx(__ldcg(plse + q) - M);
         const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sh * a.max_splits + q) * kD) + lane);
@@ -503,6 +515,327 @@ __global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(D
     }
 }
 
+// ------------------------------------------------------------------ grouped heads on tensor cores
+//
+// For G >= 4 query heads per key/value head the per-row shuffle reductions
+// above bound the kernel, not HBM.  This variant keeps the same item stream
+// (one warp per (sequence, split, key/value head) item, a 2-slot ring, the
+// same split-KV merge) but computes each 16-key tile with warp-level tensor
+// core MMAs (m16n8k16, bf16 in, fp32 accumulate): S = Q K^T with the G query
+// rows padded to 16, then O^T += V^T P^T, where the query heads are the
+// product's 8 columns (no padding for G = 8) and P^T's fragments are exactly
+// the S accumulators a lane holds.  K/V tiles arrive by TMA in
+// 128-byte-swizzled boxes so that the ldmatrix fragment loads are
+// conflict-free.
+
+constexpr int kMmaWarps = 10;
+constexpr int kScratchBytes = 8 * kD * 4;  // per warp: up to 8 unnormalised O rows (fp32)
+constexpr int kMmaSmem = kMmaWarps * (kStages * kSlotBytes + kScratchBytes) + kMmaWarps * kStages * 8 +
+                         (kMaxSmemSeqs + 1) * 4 + 64 + 1024;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D = A B + D, m16n8k16, A row-major bf16, B column-major bf16, fp32 D.
+__device__ __forceinline__ void mma_bf16_4(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// The same with rows 8..15 of A zero (the padding of the query group).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk c (0..15: dims 8c..8c+7) of tile row r in a
+// slot half (two 64-column boxes of 16 rows, 128-byte swizzle).
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+    return (uint32_t)((c >> 3) * 2048 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Lane 0: the TMA copies of tile t of `it` (K and V, 2 boxes each).
+__device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                                               uint8_t *slots, uint64_t *full, int slot, const Item &it, int t,
+                                               int phys) {
+    uint64_t *bar = full + slot;
+    if (phys < 0) {
+        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+        mbar_arrive(bar);
+        return;
+    }
+    const int tok = it.tok0 + t * kTileTok;
+    const int y = (phys * a.Hkv + it.h) * a.block_size + (tok % a.block_size);
+    uint8_t *dst = slots + slot * kSlotBytes;
+    fence_proxy_async_smem();  // the warp's generic writes to the slot (dead-row zeroing) come first
+    mbar_arrive_expect_tx(bar, kSlotBytes);
+    tma_load_2d(dst, tmK, bar, 0, y);
+    tma_load_2d(dst + 2048, tmK, bar, 64, y);
+    tma_load_2d(dst + kTileBytes, tmV, bar, 0, y);
+    tma_load_2d(dst + kTileBytes + 2048, tmV, bar, 64, y);
+}
+
+// Output of a finished grouped item: G unnormalised rows in `scratch`
+// ([G][d] fp32), row g's max / sum in lane 4g.  One fence and G parallel
+// completion counts for the whole group; rows whose last split this was are
+// merged.
+template <int G>
+__device__ __forceinline__ void finish_group(const DecodeArgs &a, int s, int h, int p, int lane,
+                                             const float *scratch, float m, float l, bool saw_bad) {
+    const int nsplit = a.item_start[s + 1] - a.item_start[s];
+    const int gl = lane & 7;  // lanes 0..G-1: the row they report
+    const float mg_l = __shfl_sync(0xffffffffu, m, 4 * gl);
+    const float lg_l = __shfl_sync(0xffffffffu, l, 4 * gl);
+    if (nsplit == 1) {
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+            const size_t sh = (size_t)s * a.H + h * G + g;
+            const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
+            const float inv = (!saw_bad && lg > 0.f) ? 1.f / lg : 0.f;
+            const float4 v = *reinterpret_cast<const float4 *>(scratch + g * kD + 4 * lane);
+            *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) =
+                make_uint2(pack_bf16x2(v.x * inv, v.y * inv), pack_bf16x2(v.z * inv, v.w * inv));
+        }
+        if (lane < G)
+            a.LSE[(size_t)s * a.H + h * G + lane] =
+                (!saw_bad && lg_l > 0.f) ? (mg_l + __log2f(lg_l)) * kLn2 : -INFINITY;
+        return;
+    }
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        const size_t pidx = ((size_t)s * a.H + h * G + g) * a.max_splits + p;
+        const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
+        const float inv = lg > 0.f ? 1.f / lg : 0.f;
+        const float4 v = *reinterpret_cast<const float4 *>(scratch + g * kD + 4 * lane);
+        *reinterpret_cast<float4 *>(a.part_o + pidx * kD + 4 * lane) =
+            make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+    }
+    if (lane < G)
+        a.part_lse[((size_t)s * a.H + h * G + lane) * a.max_splits + p] =
+            lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
+    if (lane == 0 && saw_bad) atomicOr(a.seq_bad + s, 1);
+    __threadfence();  // partials (and the bad mark) before the completion counts
+    __syncwarp();
+    bool last = false;
+    if (lane < G) last = atomicAdd(a.done_cnt + (size_t)s * a.H + h * G + lane, 1) == nsplit - 1;
+    const uint32_t lastm = __ballot_sync(0xffffffffu, last);
+    if (!lastm) return;
+    __threadfence();
+#pragma unroll 1
+    for (int g = 0; g < G; ++g)
+        if (lastm >> g & 1u) merge_row(a, s, (size_t)s * a.H + h * G + g, nsplit, lane);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      DecodeArgs a) {
+    static_assert(G == 4 || G == 8, "query group of 4 or 8");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head of the group) and column pair
+    uint8_t *slots = smem + (size_t)wid * kStages * kSlotBytes;
+    float *scratch = reinterpret_cast<float *>(smem + kMmaWarps * kStages * kSlotBytes + wid * kScratchBytes);
+    uint64_t *full =
+        reinterpret_cast<uint64_t *>(smem + kMmaWarps * (kStages * kSlotBytes + kScratchBytes)) + wid * kStages;
+    if (lane == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        for (int i = 0; i < kStages; ++i) mbar_init(full + i, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    pdl_wait();
+    const int32_t *starts = a.item_start;
+    if (a.num_seqs <= kMaxSmemSeqs) {
+        int32_t *st = reinterpret_cast<int32_t *>(smem + kMmaWarps * (kStages * kSlotBytes + kScratchBytes) +
+                                                  kMmaWarps * kStages * 8);
+        for (int i = threadIdx.x; i <= a.num_seqs; i += blockDim.x) st[i] = a.item_start[i];
+        __syncthreads();
+        starts = st;
+    }
+    const int total = starts[a.num_seqs] * a.Hkv;
+    int s_hint = 0;
+
+    Item cur, nxt;
+    fetch_item<G>(a, starts, total, lane, s_hint, cur);
+    bool have_nxt = false, exhausted = (cur.nt == 0);
+    int pq = 0, pt = 0;
+    uint32_t gi = 0, gc = 0;
+    bool dead = false;
+
+    auto produce = [&]() -> bool {
+        for (;;) {
+            const int pnt = pq ? nxt.nt : cur.nt;
+            if (pt < pnt) {
+                const int phys = pq ? tile_block(a, nxt, pt) : tile_block(a, cur, pt);
+                if (lane == 0) issue_tile_tma(a, &tmK, &tmV, slots, full, gi % kStages, pq ? nxt : cur, pt, phys);
+                __syncwarp();
+                ++pt;
+                ++gi;
+                return true;
+            }
+            if (pq == 1 || exhausted) return false;
+            fetch_item<G>(a, starts, total, lane, s_hint, nxt);
+            if (nxt.nt == 0) {
+                exhausted = true;
+                return false;
+            }
+            have_nxt = true;
+            pq = 1;
+            pt = 0;
+        }
+    };
+
+    if (!exhausted) {
+        while (gi - gc < (uint32_t)kStages && produce()) {
+        }
+    }
+    const uint32_t slots_u32 = smem_u32(slots);
+    while (cur.nt > 0) {
+        // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
+        // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
+        uint32_t qa0[8], qa2[8];
+        {
+            const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+                a.q + ((size_t)cur.s * a.H + cur.h * G + (gq < G ? gq : 0)) * kD);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qa0[ks] = gq < G ? __ldg(qrow + 8 * ks + tq) : 0u;
+                qa2[ks] = gq < G ? __ldg(qrow + 8 * ks + 4 + tq) : 0u;
+            }
+        }
+        float m = -INFINITY, l = 0.f;  // row gq: running max (log2 units) and this lane's part of the sum
+        // O^T accumulators: o[mb] holds dims 16mb + gq (0, 1) and 16mb + gq + 8
+        // (2, 3) of query heads 2tq (0, 2) and 2tq + 1 (1, 3)
+        float o[8][4];
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) o[mb][0] = o[mb][1] = o[mb][2] = o[mb][3] = 0.f;
+        bool saw_bad = false;
+        for (int t = 0; t < cur.nt; ++t) {
+            const int slot = gc % kStages;
+            if (!mbar_wait(full + slot, (gc / kStages) & 1u, a.err)) {
+                dead = true;
+                break;
+            }
+            const int tok = cur.tok0 + t * kTileTok;
+            const bool tile_ok = tile_block(a, cur, t) >= 0;
+            saw_bad |= !tile_ok;
+            if (tile_ok) {
+                const uint32_t kt = slots_u32 + slot * kSlotBytes, vt = kt + kTileBytes;
+                const int valid = min(kTileTok, cur.tok1 - tok);  // live keys of the tile (>= 1)
+                if (valid < kTileTok) {
+                    // slots past the sequence may hold anything (NaN included) and
+                    // 0 * NaN = NaN in P V: zero the dead V rows first
+                    uint8_t *vrows = slots + slot * kSlotBytes + kTileBytes;
+                    for (int e = lane; e < (kTileTok - valid) * 16; e += 32) {
+                        const int r = valid + (e >> 4), c = e & 15;
+                        *reinterpret_cast<uint4 *>(vrows + sw_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    __syncwarp();
+                }
+                // S = Q K^T: keys 0..7 (n-block 0) and 8..15 (n-block 1)
+                float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int q = lane >> 3, i = lane & 7;
+                    const int key = 8 * (q >> 1) + i;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t b00, b01, b10, b11;
+                        ldsm_x4(kt + sw_off(key, 2 * ks + (q & 1)), b00, b01, b10, b11);
+                        mma_bf16(s0, qa0[ks], qa2[ks], b00, b01);
+                        mma_bf16(s1, qa0[ks], qa2[ks], b10, b11);
+                    }
+                }
+                // online softmax of row gq over the tile's 16 keys (this lane:
+                // keys 2tq, 2tq+1, 8+2tq, 9+2tq)
+                float x[4] = {s0[0] * a.scale_log2, s0[1] * a.scale_log2, s1[0] * a.scale_log2,
+                              s1[1] * a.scale_log2};
+                const int kc[4] = {2 * tq, 2 * tq + 1, 8 + 2 * tq, 9 + 2 * tq};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (kc[e] >= valid) x[e] = -INFINITY;
+                float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m, mx);  // finite: key 0 of every tile is live
+                const float alpha = ex2_approx(m - m_new);
+                float p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[e] = ex2_approx(x[e] - m_new);
+                l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
+                m = m_new;
+                // this lane's accumulators belong to query heads 2tq and 2tq + 1
+                const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * tq);
+                const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * tq + 4);
+#pragma unroll
+                for (int mb = 0; mb < 8; ++mb) {
+                    o[mb][0] *= al0;
+                    o[mb][2] *= al0;
+                    o[mb][1] *= al1;
+                    o[mb][3] *= al1;
+                }
+                // P^T fragments (keys 2tq, 2tq + 1 and 8 + 2tq, 9 + 2tq of head gq)
+                const uint32_t pb0 = pack_bf16x2(p[0], p[1]), pb1 = pack_bf16x2(p[2], p[3]);
+                // O^T += V^T P^T: dims 16mb .. 16mb + 15 per m-block
+                {
+                    const int q = lane >> 3, i = lane & 7;
+                    const int key = 8 * (q >> 1) + i;
+#pragma unroll
+                    for (int mb = 0; mb < 8; ++mb) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t(vt + sw_off(key, 2 * mb + (q & 1)), a0, a1, a2, a3);
+                        mma_bf16_4(o[mb], a0, a1, a2, a3, pb0, pb1);
+                    }
+                }
+            }
+            ++gc;
+            __syncwarp();  // every lane is done with the slot before it is refilled
+            if (gi - gc < (uint32_t)kStages) produce();
+        }
+        if (dead) break;
+        // unnormalised O rows -> per-warp scratch, then the common finish
+        // (final row, or partial + merge by the last split)
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (2 * tq < G) {
+#pragma unroll
+            for (int mb = 0; mb < 8; ++mb) {
+                scratch[(2 * tq) * kD + 16 * mb + gq] = o[mb][0];
+                scratch[(2 * tq + 1) * kD + 16 * mb + gq] = o[mb][1];
+                scratch[(2 * tq) * kD + 16 * mb + gq + 8] = o[mb][2];
+                scratch[(2 * tq + 1) * kD + 16 * mb + gq + 8] = o[mb][3];
+            }
+        }
+        __syncwarp();
+        finish_group<G>(a, cur.s, cur.h, cur.p, lane, scratch, m, l, saw_bad);
+        __syncwarp();  // scratch reads done before the next item writes it
+        if (!have_nxt) break;
+        cur = nxt;
+        have_nxt = false;
+        pq = 0;
+        while (gi - gc < (uint32_t)kStages && produce()) {
+        }
+    }
+    if (dead && lane == 0) {
+        for (uint32_t g = gc; g < gi; ++g) mbar_wait(full + g % kStages, (g / kStages) & 1u, nullptr);
+    }
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
@@ -570,6 +903,34 @@ attn_status launch_split(const DecodeArgs &a, int dev, int sms, cudaStream_t str
     return cudaLaunchKernelEx(&cfg, decode_split_kernel<G>, a) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
+template <int G>
+attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int sms, cudaStream_t stream) {
+    static bool attr_set[64] = {false};
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(decode_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem) !=
+            cudaSuccess)
+            return ATTN_ECUDA;
+        attr_set[dev] = true;
+    }
+    const long long rows = (long long)p.num_blocks * p.Hkv * p.block_size;
+    if (rows > 0x7fffffffLL) return launch_split<G>(a, dev, sms, stream);  // TMA row coordinates are 32-bit
+    CUtensorMap tk, tv;
+    if (!make_tensor_map_2d_bf16(&tk, p.k_cache, kD, rows, kD, kTileTok) ||
+        !make_tensor_map_2d_bf16(&tv, p.v_cache, kD, rows, kD, kTileTok))
+        return ATTN_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(kMmaWarps * 32);
+    cfg.dynamicSmemBytes = kMmaSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<G>, tk, tv, a) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     static int sm_count[64] = {0};
     int dev = 0;
@@ -612,8 +973,8 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     switch (G) {
         case 1: return launch_split<1>(a, dev, sm_count[dev], stream);
         case 2: return launch_split<2>(a, dev, sm_count[dev], stream);
-        case 4: return launch_split<4>(a, dev, sm_count[dev], stream);
-        case 8: return launch_split<8>(a, dev, sm_count[dev], stream);
+        case 4: return launch_mma<4>(a, p, dev, sm_count[dev], stream);
+        case 8: return launch_mma<8>(a, p, dev, sm_count[dev], stream);
     }
     return ATTN_EUNSUPPORTED;
 }

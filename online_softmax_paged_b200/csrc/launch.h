@@ -2,6 +2,7 @@
 // kernel translation units.  Not installed; the public ABI is include/attn.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -74,6 +75,11 @@ struct Fp8Launch {
     float scale;
     int32_t *err_flag;
 };
+
+// 2-D bf16 tensor map over `rows` rows of `inner` elements (row pitch
+// `pitch_elems`), box 64 x box_rows, 128-byte swizzle (prefill_sm100.cu).
+bool make_tensor_map_2d_bf16(CUtensorMap *m, const void *base, long long inner, long long rows, long long pitch_elems,
+                             int box_rows);
 
 attn_status launch_dense_f32(const DenseLaunch &p, cudaStream_t stream);
 attn_status launch_quantize_fp8(const QuantLaunch &p, cudaStream_t stream);

@@ -987,6 +987,11 @@ attn_status launch_fp8_t(const Fp8Launch &p, cudaStream_t stream) {
 
 }  // namespace
 
+bool make_tensor_map_2d_bf16(CUtensorMap *m, const void *base, long long inner, long long rows, long long pitch_elems,
+                             int box_rows) {
+    return make_map_2d(m, base, inner, rows, pitch_elems, box_rows);
+}
+
 attn_status launch_prefill_fp8(const Fp8Launch &p, cudaStream_t stream) {
     return p.causal ? launch_fp8_t<true>(p, stream) : launch_fp8_t<false>(p, stream);
 }

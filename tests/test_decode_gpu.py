@@ -224,3 +224,29 @@ def test_gqa_decode_bad_group_rejected():
     q = torch.zeros((2, 12, 128), dtype=torch.bfloat16, device="cuda")  # group of 3
     with pytest.raises(osp.AttnError):
         osp.paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, 16)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_nan_in_unused_cache_slots_does_not_leak(G):
+    """Every cache slot no sequence uses (tails of last blocks, unused blocks)
+    set to NaN: the output equals the clean run bit for bit."""
+    osp = _osp()
+    Hkv = 32 // G
+    lens = [1, 17, 255, 300, 1000, 33, 2047]
+    p = W.paged_uniform(H=Hkv, d=128, block_size=32, pool=400, len_hi=2048, seed=50 + G, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(60 + G)
+    q = torch.randn((len(lens), 32, 128), generator=g, device="cuda").to(torch.bfloat16)
+    O1, L1 = osp.paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, 32, scale=p.scale)
+    live = torch.zeros(p.k_cache.shape[0], 32, dtype=torch.bool)
+    t, sl = p.block_table.cpu(), p.seq_lens.cpu()
+    for s in range(t.shape[0]):
+        L = int(sl[s])
+        for lb in range(-(-L // 32)):
+            live[int(t[s, lb]), :min(32, L - lb * 32)] = True
+    dead = (~live).to("cuda")[:, None, :, None]
+    kc = p.k_cache.clone().masked_fill_(dead, float("nan"))
+    vc = p.v_cache.clone().masked_fill_(dead, float("nan"))
+    O2, L2 = osp.paged_attn_decode_gqa(q, kc, vc, p.block_table, p.seq_lens, 32, scale=p.scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(O2.float()).all()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
