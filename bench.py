@@ -24,8 +24,10 @@ pairs) (causal: N(N+1)/2 per head); decode bytes = K/V bytes the sequences
 attend over (sum_s L_s * 2 * H * d * 2; for the shared-prefix workload the
 unique physical bytes, logical bytes reported beside).
 
-Timing: W untimed warm-up steps, then K steps between barrier +
-cuda.synchronize, CUDA events on the launching stream around every launch;
+Timing: W untimed warm-up steps, then the K steps captured once in a CUDA
+graph and replayed between barrier + cuda.synchronize, CUDA events on the
+launching stream around the replay (device time of K back-to-back steps;
+--eager times K separate calls with events around each instead);
 inputs rotate over copies whose total exceeds L2 (prefill) or exceed it alone
 (decode pools of GB).  Multi-GPU (torchrun): every rank runs its own replica
 (independent problems, weak scaling, no collective on the data path); the
@@ -572,6 +574,12 @@ class Fp8Prefill:
             e1.record(st)
             self.kernel_events.append((e0, e1))
 
+    def dominant(self, i, osp):
+        """The attention launch alone (on the codes the last quantisation left)."""
+        s = self.sets[i % self.copies]
+        osp.attn_fwd_fp8(self.q8, self.qs, self.k8, self.ks, s["V"], O=self.O, LSE=self.LSE, causal=True,
+                         scale=s["scale"])
+
     def config(self):
         return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N, "d": self.d, "causal": True,
                 "dtype": "e4m3 Q/K, bf16 V/P/O", "global_batch": self.B, "seq_len": self.N,
@@ -768,14 +776,75 @@ def make_workload(name, device, seed=0):
 
 # ---------------------------------------------------------------- timing
 
-def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0):
+def time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s=0.0):
+    """The K timed steps captured once into a CUDA graph and replayed between
+    barrier + synchronize, CUDA events around the replay: device time of K
+    back-to-back steps, without the host's per-call launch cost (a serving
+    loop replays its decode steps the same way).  Steps of several launches
+    whose roofline is one kernel's also get a graph of that kernel alone.
+    Returns (per-step or per-kernel ms list, total ms, wall s)."""
+    st = torch.cuda.current_stream(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            wl.step(warmup + i, osp)
+    gk = None
+    if hasattr(wl, "dominant"):
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gk):
+            for i in range(steps):
+                wl.dominant(warmup + i, osp)
+    g.replay()  # first replay uploads the graph
+    if gk is not None:
+        gk.replay()
+    torch.cuda.synchronize(device)
+    # the soak replays the same graph right before the timed replay, so the
+    # timed steps run at the clocks a loaded GPU settles to (capturing left
+    # the GPU idle)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < soak_s:
+        g.replay()
+        torch.cuda.synchronize(device)
+    barrier(ws)
+    torch.cuda.synchronize(device)
+    t_region0 = time.perf_counter()
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(st)
+    g.replay()
+    g1.record(st)
+    torch.cuda.synchronize(device)
+    barrier(ws)
+    wall = time.perf_counter() - t_region0
+    total_ms = g0.elapsed_time(g1)
+    per = [total_ms / steps] * steps
+    if gk is not None:
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        k0.record(st)
+        gk.replay()
+        k1.record(st)
+        torch.cuda.synchronize(device)
+        per = [k0.elapsed_time(k1) / steps] * steps
+    del g, gk
+    return per, total_ms, wall
+
+
+def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0, graph=False):
     """W warm-up steps, an optional untimed soak (so the clocks sampled
     around the timed region reflect a loaded GPU), then K timed steps between
-    barrier + synchronize with CUDA events around every launch."""
+    barrier + synchronize with CUDA events around every launch (or, with
+    ``graph``, around one replay of the K steps captured in a CUDA graph)."""
     st = torch.cuda.current_stream(device)
     for i in range(warmup):
         wl.step(i, osp)
     torch.cuda.synchronize(device)
+    if graph:
+        try:
+            return time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s) + ("graph",)
+        except Exception as e:  # capture unsupported here: time eagerly
+            print(f"CUDA graph capture failed ({e!r}); timing eagerly", file=sys.stderr)
+            torch.cuda.synchronize(device)
     if soak_s > 0:
         t0, i = time.perf_counter(), 0
         while time.perf_counter() - t0 < soak_s:
@@ -806,7 +875,7 @@ def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0):
         wl.record = False
         per = [a.elapsed_time(b) for a, b in wl.kernel_events]
     total_ms = g0.elapsed_time(g1)
-    return per, total_ms, wall
+    return per, total_ms, wall, "eager"
 
 
 def roofline(wl, per_ms, pk, pk_src, bound, clocks=None):
@@ -857,7 +926,8 @@ def run_ours(args):
     bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill, Fp8Prefill)) else "hbm"
     with ClockSampler(local) as clocks:
         t_load0 = time.perf_counter()
-        per, total_ms, wall = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak)
+        per, total_ms, wall, timing = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak,
+                                                 graph=not args.eager)
         t_load1 = time.perf_counter()
     t_max = max_over_ranks(total_ms, ws)
     work_all = sum_over_ranks(wl.work * args.steps, ws)
@@ -872,12 +942,14 @@ def run_ours(args):
     extra = {}
     if args.workload == "prefill_2k" and not args.no_decode:
         dec = make_workload("decode_uniform", device, seed=args.seed + rank)
-        per_d, total_d, _ = time_steps(dec, osp, args.steps, args.warmup, device, ws, soak_s=min(args.soak, 0.5))
+        per_d, total_d, _, timing_d = time_steps(dec, osp, args.steps, args.warmup, device, ws,
+                                                 soak_s=min(args.soak, 0.5), graph=not args.eager)
         td = max_over_ranks(total_d, ws)
         extra["decode"] = {"workload": "decode_uniform", "value": round(sum_over_ranks(dec.work * args.steps, ws)
                                                                         / (td * 1e-3) / 1e9, 2),
                            "unit": "GB/s", "ms_per_step": round(td / args.steps, 5),
-                           "roofline": roofline(dec, per_d, pk, pk_src, "hbm"), "config": dec.config(),
+                           "roofline": roofline(dec, per_d, pk, pk_src, "hbm"),
+                           "config": {**dec.config(), "timing": timing_d},
                            "gpu_launches": dec.launches_per_step * args.steps}
         del dec
 
@@ -892,7 +964,7 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16" if isinstance(wl, Fp8Prefill) else "bf16",
                 "data": "synthetic (seeded N(0,1), bf16)",
-                "config": {**wl.config(), "parallelism": f"replicas{ws}" if ws > 1 else "single"},
+                "config": {**wl.config(), "parallelism": f"replicas{ws}" if ws > 1 else "single", "timing": timing},
                 "roofline": rl, "cpu_baseline": cpu,
                 "e2e": {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
@@ -1034,6 +1106,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode leg of the default line")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing (clocks)")
+    ap.add_argument("--eager", action="store_true",
+                    help="time K eager calls instead of one replay of the K steps captured in a CUDA graph")
     args = ap.parse_args(argv)
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps

@@ -102,13 +102,13 @@ def attn_status_str(status: int) -> str:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
-    return ctypes.c_void_p(stream.cuda_stream)
+    return stream.cuda_stream
 
 
 def _check_cuda(*ts):
@@ -234,8 +234,8 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=
         LSE = torch.empty((S, H), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    need = paged_attn_decode_workspace_size(S, H, d, mb, block_size)
-    if workspace is None:
+    if workspace is None:  # (a given workspace is checked against the need by the library)
+        need = paged_attn_decode_workspace_size(S, H, d, mb, block_size)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = load().paged_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                   int(block_size), _ptr(O), _ptr(LSE), S, H, d, num_blocks, mb, float(scale),
@@ -267,8 +267,8 @@ def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     mb = block_table.shape[1]
-    need = paged_attn_decode_workspace_size(S, Hq, d, mb, block_size)
-    if workspace is None:
+    if workspace is None:  # (a given workspace is checked against the need by the library)
+        need = paged_attn_decode_workspace_size(S, Hq, d, mb, block_size)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = load().paged_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                       int(block_size), _ptr(O), _ptr(LSE), S, Hq, Hkv, d, nb, mb, float(scale),

@@ -588,6 +588,59 @@ __device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtens
     tma_load_2d(dst + kTileBytes + 2048, tmV, bar, 64, y);
 }
 
+// The final rows of query heads sh0 .. sh0 + G - 1 of sequence s (those set
+// in `mask`) from their nsplit partials: every row's loads of split q go out
+// together, so the G rows share the latency of one (the same per-row
+// arithmetic order as merge_row).
+template <int G>
+__device__ __forceinline__ void merge_rows(const DecodeArgs &a, int s, size_t sh0, int nsplit, int lane,
+                                           uint32_t mask) {
+    if (__ldcg(a.seq_bad + s)) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            if (mask >> g & 1u) {
+                *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) = make_uint2(0u, 0u);
+                if (lane == 0) a.LSE[sh0 + g] = -INFINITY;
+            }
+        return;
+    }
+    float M[G], tot[G];
+    float4 acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) M[g] = -INFINITY;
+#pragma unroll 2
+    for (int q = 0; q < nsplit; ++q)
+#pragma unroll
+        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(a.part_lse + (sh0 + g) * a.max_splits + q));
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        tot[g] = 0.f;
+        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll 2
+    for (int q = 0; q < nsplit; ++q) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const size_t pidx = (sh0 + g) * a.max_splits + q;
+            const float w = ex2_approx(__ldcg(a.part_lse + pidx) - M[g]);
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + pidx * kD) + lane);
+            tot[g] += w;
+            acc[g].x = fmaf(w, v.x, acc[g].x);
+            acc[g].y = fmaf(w, v.y, acc[g].y);
+            acc[g].z = fmaf(w, v.z, acc[g].z);
+            acc[g].w = fmaf(w, v.w, acc[g].w);
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        if (!(mask >> g & 1u)) continue;
+        const float inv = tot[g] > 0.f ? 1.f / tot[g] : 0.f;
+        *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) =
+            make_uint2(pack_bf16x2(acc[g].x * inv, acc[g].y * inv), pack_bf16x2(acc[g].z * inv, acc[g].w * inv));
+        if (lane == 0) a.LSE[sh0 + g] = tot[g] > 0.f ? (M[g] + __log2f(tot[g])) * kLn2 : -INFINITY;
+    }
+}
+
 // Output of a finished grouped item: G unnormalised rows in `scratch`
 // ([G][d] fp32), row g's max / sum in lane 4g.  One fence and G parallel
 // completion counts for the whole group; rows whose last split this was are
@@ -634,9 +687,7 @@ __device__ __forceinline__ void finish_group(const DecodeArgs &a, int s, int h, 
     const uint32_t lastm = __ballot_sync(0xffffffffu, last);
     if (!lastm) return;
     __threadfence();
-#pragma unroll 1
-    for (int g = 0; g < G; ++g)
-        if (lastm >> g & 1u) merge_row(a, s, (size_t)s * a.H + h * G + g, nsplit, lane);
+    merge_rows<G>(a, s, (size_t)s * a.H + h * G, nsplit, lane, lastm);
 }
 
 template <int G>
