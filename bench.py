@@ -303,8 +303,8 @@ class Decode:
         self.O = torch.empty_like(self.p.q)
         self.LSE = torch.empty(self.p.q.shape[:2], dtype=torch.float32, device=device)
         import online_softmax_paged_b200 as osp
-        n = osp.paged_attn_decode_workspace_size(self.p.num_seqs, self.p.H, self.p.d, self.p.max_blocks_per_seq,
-                                                 self.p.block_size)
+        n = osp.paged_attn_decode_gqa_workspace_size(self.p.num_seqs, self.p.H, self.p.k_cache.shape[1], self.p.d,
+                                                     self.p.max_blocks_per_seq, self.p.block_size)
         self.ws = torch.empty(n, dtype=torch.uint8, device=device)
         self.ws_bytes = n
         self.unit, self.scale_unit = "GB/s", 1e9

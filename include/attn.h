@@ -99,6 +99,16 @@ ATTN_API size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int
                                         int block_size);
 
 /*
+ * Bytes of device workspace paged_attn_decode_gqa needs (H_q query heads over
+ * H_kv key/value heads).  Returns 0 for invalid sizes (H_q not a multiple of
+ * H_kv, or as paged_attn_decode_workspace_size).  The partials are per query
+ * head, so it currently equals paged_attn_decode_workspace_size(num_seqs,
+ * H_q, ...); callers of paged_attn_decode_gqa should size with this one.
+ */
+ATTN_API size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int H_q, int H_kv, int d,
+                                                     int max_blocks_per_seq, int block_size);
+
+/*
  * Tokens per split-KV chunk the decode uses for these sizes (a function of
  * the sizes only, never of the data; exposed for tests and tooling).
  */
@@ -149,7 +159,7 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
  * q, O         : [num_seqs, H_q, d] bf16;   LSE : [num_seqs, H_q] fp32.
  * k_cache,
  * v_cache      : [num_blocks, H_kv, block_size, d] bf16.
- * workspace    : paged_attn_decode_workspace_size(num_seqs, H_q, d, ...) bytes.
+ * workspace    : paged_attn_decode_gqa_workspace_size(num_seqs, H_q, H_kv, d, ...) bytes.
  * Supported    : H_q / H_kv in {1, 2, 4, 8}; otherwise as paged_attn_decode
  *                (whose behaviour, checks and determinism apply unchanged;
  *                paged_attn_decode is this call with H_kv = H_q).

@@ -18,7 +18,7 @@ __all__ = [
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
     "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
-    "attn_quantize_fp8", "attn_fwd_fp8",
+    "attn_quantize_fp8", "attn_fwd_fp8", "paged_attn_decode_gqa_workspace_size",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,8 @@ ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_INDEX = 1, 2, 4, 8
 
 # every function include/attn.h declares
-EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_split_tokens",
+EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_decode_gqa_workspace_size",
+                    "paged_attn_decode_split_tokens",
                     "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_attn_prefill",
                     "attn_quantize_fp8", "attn_fwd_fp8",
                     "paged_kv_append",
@@ -66,6 +67,8 @@ def load():
     lib.attn_fwd.restype = c_int
     lib.paged_attn_decode_workspace_size.argtypes = [c_int] * 5
     lib.paged_attn_decode_workspace_size.restype = c_size
+    lib.paged_attn_decode_gqa_workspace_size.argtypes = [c_int] * 6
+    lib.paged_attn_decode_gqa_workspace_size.restype = c_size
     lib.paged_attn_decode_split_tokens.argtypes = [c_int] * 5
     lib.paged_attn_decode_split_tokens.restype = c_int
     lib.paged_attn_decode.argtypes = [vp, vp, vp, vp, vp, c_int, vp, fp, c_int, c_int, c_int, c_int, c_int,
@@ -206,6 +209,11 @@ def paged_attn_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq, block_s
     return int(load().paged_attn_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq, block_size))
 
 
+def paged_attn_decode_gqa_workspace_size(num_seqs, H_q, H_kv, d, max_blocks_per_seq, block_size) -> int:
+    return int(load().paged_attn_decode_gqa_workspace_size(int(num_seqs), int(H_q), int(H_kv), int(d),
+                                                           int(max_blocks_per_seq), int(block_size)))
+
+
 def paged_attn_decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size) -> int:
     return int(load().paged_attn_decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size))
 
@@ -268,7 +276,7 @@ def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size
         scale = 1.0 / math.sqrt(d)
     mb = block_table.shape[1]
     if workspace is None:  # (a given workspace is checked against the need by the library)
-        need = paged_attn_decode_workspace_size(S, Hq, d, mb, block_size)
+        need = paged_attn_decode_gqa_workspace_size(S, Hq, Hkv, d, mb, block_size)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = load().paged_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                       int(block_size), _ptr(O), _ptr(LSE), S, Hq, Hkv, d, nb, mb, float(scale),

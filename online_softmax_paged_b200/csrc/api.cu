@@ -61,13 +61,21 @@ attn_status attn_fwd_fp8(const void *q8, const float *q_scale, const void *k8, c
 size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq, int block_size) {
     if (num_seqs < 0 || H < 1 || d != 128 || max_blocks_per_seq < 1 || block_size < 16 || block_size % 16)
         return 0;
-    return osp::decode_workspace_bytes(num_seqs, H, d, max_blocks_per_seq, block_size);
+    return osp::decode_workspace_bytes(num_seqs, H, H, d, max_blocks_per_seq, block_size);
+}
+
+size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int H_q, int H_kv, int d, int max_blocks_per_seq,
+                                            int block_size) {
+    if (num_seqs < 0 || H_q < 1 || H_kv < 1 || H_q % H_kv || d != 128 || max_blocks_per_seq < 1 ||
+        block_size < 16 || block_size % 16)
+        return 0;
+    return osp::decode_workspace_bytes(num_seqs, H_q, H_kv, d, max_blocks_per_seq, block_size);
 }
 
 int paged_attn_decode_split_tokens(int num_seqs, int H, int d, int max_blocks_per_seq, int block_size) {
     if (num_seqs < 0 || H < 1 || d != 128 || max_blocks_per_seq < 1 || block_size < 16 || block_size % 16)
         return 0;
-    return osp::decode_split_tokens(num_seqs, H, d, max_blocks_per_seq, block_size);
+    return osp::decode_split_tokens(num_seqs, H, H, d, max_blocks_per_seq, block_size);
 }
 
 namespace {
@@ -93,7 +101,7 @@ attn_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
         return ATTN_EINVAL;
     if (((uintptr_t)block_table & 3u) || ((uintptr_t)seq_lens & 3u) || ((uintptr_t)LSE & 3u)) return ATTN_EINVAL;
     if ((long long)num_seqs * H > 0x7fffffffLL / 4) return ATTN_EINVAL;
-    if (workspace_bytes < osp::decode_workspace_bytes(num_seqs, H, d, max_blocks_per_seq, block_size))
+    if (workspace_bytes < osp::decode_workspace_bytes(num_seqs, H, Hkv, d, max_blocks_per_seq, block_size))
         return ATTN_EINVAL;
     osp::DecodeLaunch p{q,        k_cache,  v_cache, block_table, seq_lens,         O,          LSE,
                         num_seqs, H,        d,       num_blocks,  max_blocks_per_seq, block_size, scale,

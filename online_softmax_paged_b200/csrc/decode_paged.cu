@@ -907,10 +907,14 @@ WsLayout ws_layout(int num_seqs, int H, int max_splits) {
 
 }  // namespace
 
-int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_size) {
+int decode_split_tokens(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size) {
     (void)d;
     const long long max_len = (long long)max_blocks * block_size;
     const long long work = (long long)num_seqs * H * max_len;
+    // (the grouping does not change the split: half-length splits for groups
+    // of 4 and 8, which would double the items, measured slower -- more
+    // partials, fences and merges than the tail they save)
+    (void)Hkv;
     long long split = 256;
     // larger splits for large problems (bounded workspace), at most 64 blocks
     // per split (the kernel keeps a split's block ids in two registers per lane)
@@ -918,14 +922,14 @@ int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_si
     return (int)split;
 }
 
-int decode_max_splits(int num_seqs, int H, int d, int max_blocks, int block_size) {
+int decode_max_splits(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size) {
     const long long max_len = (long long)max_blocks * block_size;
-    const int split = decode_split_tokens(num_seqs, H, d, max_blocks, block_size);
+    const int split = decode_split_tokens(num_seqs, H, Hkv, d, max_blocks, block_size);
     return (int)((max_len + split - 1) / split);
 }
 
-size_t decode_workspace_bytes(int num_seqs, int H, int d, int max_blocks, int block_size) {
-    const int ms = decode_max_splits(num_seqs, H, d, max_blocks, block_size);
+size_t decode_workspace_bytes(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size) {
+    const int ms = decode_max_splits(num_seqs, H, Hkv, d, max_blocks, block_size);
     return ws_layout(num_seqs, H, ms < 1 ? 1 : ms).total;
 }
 
@@ -1006,8 +1010,8 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.num_blocks = p.num_blocks;
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
-    a.split_tokens = decode_split_tokens(p.num_seqs, p.H, p.d, p.max_blocks, p.block_size);
-    a.max_splits = decode_max_splits(p.num_seqs, p.H, p.d, p.max_blocks, p.block_size);
+    a.split_tokens = decode_split_tokens(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
+    a.max_splits = decode_max_splits(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
     if (a.max_splits < 1) a.max_splits = 1;
     a.scale_log2 = p.scale * 1.4426950408889634f;
     const WsLayout w = ws_layout(p.num_seqs, p.H, a.max_splits);

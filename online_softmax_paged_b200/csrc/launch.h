@@ -90,8 +90,9 @@ attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream);
 attn_status launch_prefill_bf16(const DenseLaunch &p, cudaStream_t stream);
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream);
 
-int decode_split_tokens(int num_seqs, int H, int d, int max_blocks, int block_size);
-int decode_max_splits(int num_seqs, int H, int d, int max_blocks, int block_size);
-size_t decode_workspace_bytes(int num_seqs, int H, int d, int max_blocks, int block_size);
+// H query heads over Hkv key/value heads (Hkv = H: multi-head)
+int decode_split_tokens(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size);
+int decode_max_splits(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size);
+size_t decode_workspace_bytes(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size);
 
 }  // namespace osp

@@ -119,3 +119,13 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         osp.attn_fwd(x, x, x)
+
+
+def test_gqa_workspace_size(lib):
+    """Grouped workspace: partials are per query head, so it equals the
+    multi-head size for every valid grouping; invalid groupings give 0."""
+    mha = osp.paged_attn_decode_workspace_size(64, 32, 128, 256, 16)
+    for hkv in (32, 16, 8, 4):
+        assert osp.paged_attn_decode_gqa_workspace_size(64, 32, hkv, 128, 256, 16) == mha
+    assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 3, 128, 256, 16) == 0
+    assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 0, 128, 256, 16) == 0
