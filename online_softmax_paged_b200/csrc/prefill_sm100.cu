@@ -233,7 +233,7 @@ __device__ __forceinline__ int snake_unit(int r, int c, int G, int n_units) {
 }
 
 // Unit u of the kernel's unit space -> UnitInfo.  Dense units are numbered
-// longest first when causal; paged units as (query block, sequence, head)
+// longest first when causal; paged units as (sequence, query block, head)
 // with later query blocks (more keys) first.  A paged unit past its
 // sequence's new tokens, or of an inconsistent sequence, gets n0 = n1 = 0;
 // the latter also gets `bad` (cu_q outside [0, total_q] or decreasing:
@@ -252,10 +252,15 @@ __device__ __forceinline__ void get_unit(const PrefillArgs &a, bool causal, int 
         x.pos0 = 0;
         x.qtok0 = 0;
     } else {
-        const int SH = a.S * a.Hq;
-        const int qb = a.nqb - 1 - u / SH, rem = u % SH;
-        x.s = rem / a.Hq;
-        x.head = rem - x.s * a.Hq;
+        // sequence-major, so that the CTAs at work at any time share one or
+        // two sequences' K/V in L2; within a sequence the later (longer)
+        // query blocks first, then the query heads (a key/value head's group
+        // adjacent)
+        const int per_seq = a.nqb * a.Hq;
+        x.s = u / per_seq;
+        const int rem = u - x.s * per_seq;
+        const int qb = a.nqb - 1 - rem / a.Hq;
+        x.head = rem - (rem / a.Hq) * a.Hq;
         x.kv_head = x.head / (a.Hq / a.Hkv);
         x.qtok0 = a.cu_q[x.s];
         x.nq = a.cu_q[x.s + 1] - x.qtok0;
