@@ -168,7 +168,10 @@ class ClockSampler:
 
 
 KERNEL_SOURCES = {"prefill_bf16_kernel": ("prefill_sm100.cu", "ptx.cuh", "launch.h"),
-                  "decode_split_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h")}
+                  "decode_split_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h"),
+                  "decode_mma_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h"),
+                  "kv_append_kernel": ("kv_cache_ops.cu", "ptx.cuh", "launch.h"),
+                  "block_copy_kernel": ("kv_cache_ops.cu", "ptx.cuh", "launch.h")}
 
 
 def kernel_sources_hash(kernel: str) -> str:
@@ -309,7 +312,10 @@ class Decode:
         self.ws_bytes = n
         self.unit, self.scale_unit = "GB/s", 1e9
         self.launches_per_step = 2
-        self.kernel = "decode_split_kernel"  # timed with its plan kernel: the events wrap the whole call
+        # timed with its plan kernel (the events wrap the whole call); groups of
+        # 4 and 8 run the tensor-core variant
+        G = self.p.q.shape[1] // self.p.k_cache.shape[1]
+        self.kernel = "decode_mma_kernel" if G >= 4 else "decode_split_kernel"
 
     def step(self, i, osp):
         p = self.p
