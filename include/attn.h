@@ -160,7 +160,10 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
  * k_cache,
  * v_cache      : [num_blocks, H_kv, block_size, d] bf16.
  * workspace    : paged_attn_decode_gqa_workspace_size(num_seqs, H_q, H_kv, d, ...) bytes.
- * Supported    : H_q / H_kv in {1, 2, 4, 8}; otherwise as paged_attn_decode
+ * Supported    : H_q / H_kv in {1, 2, 4} or a multiple of 8 (multi-query
+ *                attention included: groups above 8 run as groups of 8
+ *                sharing a key/value head, whose tiles are then read from
+ *                L2 after the first); otherwise as paged_attn_decode
  *                (whose behaviour, checks and determinism apply unchanged;
  *                paged_attn_decode is this call with H_kv = H_q).
  */

@@ -257,7 +257,8 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=
 def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size, O=None, LSE=None, scale=None,
                           workspace=None, err_flag=None, stream=None):
     """Grouped-query paged decode: q [S, H_q, d], caches [num_blocks, H_kv,
-    block_size, d] with H_q / H_kv in {1, 2, 4, 8}.  See include/attn.h."""
+    block_size, d] with H_q / H_kv in {1, 2, 4} or a multiple of 8 (H_kv = 1:
+    multi-query attention).  See include/attn.h."""
     _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, workspace, err_flag)
     S, Hq, d = q.shape
     nb, Hkv, bs, dk = k_cache.shape

@@ -88,7 +88,7 @@ attn_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (num_seqs < 0 || H < 1 || Hkv < 1 || num_blocks < 1 || max_blocks_per_seq < 1) return ATTN_EINVAL;
     if (H % Hkv) return ATTN_EINVAL;
     const int G = H / Hkv;
-    if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_EUNSUPPORTED;
+    if (G != 1 && G != 2 && G != 4 && G % 8 != 0) return ATTN_EUNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_EINVAL;
     if (dt != ATTN_BF16) return ATTN_EUNSUPPORTED;
     if (d != 128) return ATTN_EUNSUPPORTED;

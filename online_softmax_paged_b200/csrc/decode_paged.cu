@@ -79,7 +79,9 @@ struct DecodeArgs {
     float *part_lse;      // [num_seqs, H, max_splits] log2 units
     float *part_o;        // [num_seqs, H, max_splits, d] normalised
     int num_seqs, H, num_blocks, max_blocks, block_size, split_tokens, max_splits;
-    int Hkv;              // key/value heads; H (query heads) = Hkv * G
+    int Hkv;              // key/value heads of the item space; H (query heads) = Hkv * G
+    int kv_heads;         // key/value heads of the cache (= Hkv, or Hkv / kv_div)
+    int kv_div;           // groups above 8 run as kv_div groups of 8 per cache head
     float scale_log2;     // scale * log2(e)
 };
 
@@ -578,7 +580,7 @@ __device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtens
         return;
     }
     const int tok = it.tok0 + t * kTileTok;
-    const int y = (phys * a.Hkv + it.h) * a.block_size + (tok % a.block_size);
+    const int y = (phys * a.kv_heads + it.h / a.kv_div) * a.block_size + (tok % a.block_size);
     uint8_t *dst = slots + slot * kSlotBytes;
     fence_proxy_async_smem();  // the warp's generic writes to the slot (dead-row zeroing) come first
     mbar_arrive_expect_tx(bar, kSlotBytes);
@@ -967,8 +969,9 @@ attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int 
             return ATTN_ECUDA;
         attr_set[dev] = true;
     }
-    const long long rows = (long long)p.num_blocks * p.Hkv * p.block_size;
-    if (rows > 0x7fffffffLL) return launch_split<G>(a, dev, sms, stream);  // TMA row coordinates are 32-bit
+    const long long rows = (long long)p.num_blocks * a.kv_heads * p.block_size;
+    if (rows > 0x7fffffffLL)  // TMA row coordinates are 32-bit
+        return a.kv_div > 1 ? ATTN_EUNSUPPORTED : launch_split<G>(a, dev, sms, stream);
     CUtensorMap tk, tv;
     if (!make_tensor_map_2d_bf16(&tk, p.k_cache, kD, rows, kD, kTileTok) ||
         !make_tensor_map_2d_bf16(&tv, p.v_cache, kD, rows, kD, kTileTok))
@@ -1007,6 +1010,8 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.num_seqs = p.num_seqs;
     a.H = p.H;
     a.Hkv = p.Hkv;
+    a.kv_heads = p.Hkv;
+    a.kv_div = 1;
     a.num_blocks = p.num_blocks;
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
@@ -1030,6 +1035,15 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
         case 2: return launch_split<2>(a, dev, sm_count[dev], stream);
         case 4: return launch_mma<4>(a, p, dev, sm_count[dev], stream);
         case 8: return launch_mma<8>(a, p, dev, sm_count[dev], stream);
+    }
+    if (G % 8 == 0) {
+        // larger groups (multi-query attention): each cache head serves G / 8
+        // virtual key/value heads of 8 query heads; the items of one cache
+        // head are consecutive in the work queue, so its tiles are re-read
+        // from L2
+        a.kv_div = G / 8;
+        a.Hkv = p.H / 8;
+        return launch_mma<8>(a, p, dev, sm_count[dev], stream);
     }
     return ATTN_EUNSUPPORTED;
 }

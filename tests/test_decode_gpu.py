@@ -250,3 +250,28 @@ def test_nan_in_unused_cache_slots_does_not_leak(G):
     torch.cuda.synchronize()
     assert torch.isfinite(O2.float()).all()
     assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs", [(32, 1, 16), (32, 2, 32), (64, 4, 16)])
+def test_mqa_large_groups_full(Hq, Hkv, bs):
+    """Groups above 8 (multi-query attention at H_kv = 1): 32 or 64 query
+    heads over 1, 2 or 4 key/value heads against the grouped oracle, edge
+    lengths included; a placement shuffle is bit-identical."""
+    osp = _osp()
+    lens = [0, 1, 17, 255, 256, 257, 1000, 3000, 33]
+    p = W.paged_uniform(H=Hkv, d=128, block_size=bs, pool=1200, len_hi=3000, seed=70 + Hq + Hkv, device="cuda",
+                        lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(80 + Hkv)
+    q = torch.randn((len(lens), Hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = osp.paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, bs, scale=p.scale,
+                                       err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    O_ref, L_ref = oracle.paged_decode(to64(q), DeviceCache(p.k_cache), DeviceCache(p.v_cache),
+                                       p.block_table.cpu().numpy(), p.seq_lens.cpu().numpy(), bs, p.scale)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"mqa Hq={Hq} Hkv={Hkv} bs={bs}")
+    p2 = W.shuffle_placement(p, seed=5)
+    O2, L2 = osp.paged_attn_decode_gqa(q, p2.k_cache, p2.v_cache, p2.block_table, p2.seq_lens, bs, scale=p.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
