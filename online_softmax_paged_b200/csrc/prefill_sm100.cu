@@ -65,9 +65,10 @@ struct Cfg {
     static constexpr int kStages = D == 128 ? 4 : 8;
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = NQ * kTileBytes;
-    // one 64-column O box per query tile, staged for the TMA store
+    // one O tile (D / 64 boxes of 64 columns) staged for the TMA store, shared
+    // by the two query tiles in unit order
     static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
-    static constexpr int kBarOff = kStageOff + NQ * kBoxBytes;
+    static constexpr int kBarOff = kStageOff + kBoxes * kBoxBytes;
     // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], done,
     // stg_full[2], stg_free[2]
     static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 1 + 2 + 2;
@@ -303,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *p_full = s_full + 2;
     uint64_t *o_full = p_full + 2;
     uint64_t *done_bar = o_full + 2;
-    uint64_t *stg_full = done_bar + 1;  // the tile's 128 rows are in its staging box
-    uint64_t *stg_free = stg_full + 2;  // the TMA store has read the staging box
+    uint64_t *stg_full = done_bar + 1;  // [tile] the tile's 128 rows are in the staging buffer
+    uint64_t *stg_free = stg_full + 2;  // [0] the last TMA store has read the staging buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMiscOff + 8);
 
@@ -614,13 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_tm = tmem + lane_off + 2 * BN + i * 128;
         bool ok = true;
         uint32_t itc = 0;        // key-tile iterations done by this query tile so far
-        uint32_t stg_count = 0;  // O boxes staged by this warpgroup so far
+        uint32_t stg_count = 0;  // O tiles staged by this warpgroup so far
+        uint32_t ticket = 0;     // O tiles staged by both warpgroups before the current unit
         for (int rr = 0; ok; ++rr) {
             const int u = snake_unit(rr, c, G, n_units);
             if (u < 0) break;
             UnitInfo x;
             get_unit<PAGED>(a, CAUSAL, u, x);
             const int my_nkv = i ? x.n1 : x.n0;
+            // the staging buffer goes to the unit's tiles in order, tile 0 first;
+            // both warpgroups derive the same sequence of owners
+            const bool staged0 = x.n0 > 0 && (!PAGED || x.qrow0 + BM <= x.nq);
+            const bool staged1 = x.n1 > 0 && (!PAGED || x.qrow0 + 2 * BM <= x.nq);
+            const uint32_t my_ticket = ticket + ((i == 1 && staged0) ? 1u : 0u);
+            ticket += (staged0 ? 1u : 0u) + (staged1 ? 1u : 0u);
             const int tile_pos = x.pos0 + x.qrow0 + i * BM;  // key position of the tile's row 0
             const int row = x.qrow0 + i * BM + r_in;        // query row in the sequence
             // FP8: the dequantisation scales of this query tile and of each key
@@ -719,52 +727,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               : ((size_t)x.head * a.N + (live ? row : 0));
                 const int tile_row0 = x.qrow0 + i * BM;
                 if (!PAGED || tile_row0 + BM <= x.nq) {
-                    // Each thread writes its row into the tile's 128B-swizzled
-                    // staging box, 64 columns at a time, and one thread stores
-                    // the box with TMA (whole 128-byte row segments instead of
-                    // 32 rows per store instruction; rows past the end of a
-                    // dense sequence are clipped by the tensor map).
-                    const uint32_t stg = smem_base + C::kStageOff + i * kBoxBytes;
-                    const uint32_t row_addr = stg + r_in * 128;
+                    // The whole O tile goes, packed to bf16, into the 128B-swizzled
+                    // staging buffer (one box per 64 columns), and one thread stores
+                    // it with TMA (whole 128-byte row segments instead of 32 rows
+                    // per store instruction; rows past the end of a dense sequence
+                    // are clipped by the tensor map).  The buffer is taken in
+                    // ticket order: the previous owner's store must have read it.
+                    const uint32_t row_addr = smem_base + C::kStageOff + r_in * 128;
                     const bool issuer = quarter == 0 && lane == 0;
+                    uint32_t pk[D / 64][32];
 #pragma unroll
-                    for (int h = 0; h < D / 64 && ok; ++h) {
+                    for (int h = 0; h < D / 64; ++h) {
                         uint32_t o0[32], o1[32];
                         tmem_ld32(o_tm + 64 * h, o0);
                         tmem_ld32(o_tm + 64 * h + 32, o1);
                         tmem_wait_ld();
-                        uint32_t pk[32];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            pk[e] = pack_bf16x2(__uint_as_float(o0[2 * e]) * inv, __uint_as_float(o0[2 * e + 1]) * inv);
-                            pk[16 + e] =
+                            pk[h][e] =
+                                pack_bf16x2(__uint_as_float(o0[2 * e]) * inv, __uint_as_float(o0[2 * e + 1]) * inv);
+                            pk[h][16 + e] =
                                 pack_bf16x2(__uint_as_float(o1[2 * e]) * inv, __uint_as_float(o1[2 * e + 1]) * inv);
                         }
-                        if (stg_count > 0) {
-                            ok = wait_or_abort(&stg_free[i], (stg_count - 1) & 1, a.err, abort_flag);
-                            if (!ok) break;
-                        }
+                    }
+                    if (my_ticket > 0) {
+                        ok = wait_or_abort(&stg_free[0], (my_ticket - 1) & 1, a.err, abort_flag);
+                        if (!ok) break;
+                    }
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h)
 #pragma unroll
                         for (int ch = 0; ch < 8; ++ch)
-                            st_shared_v4(row_addr + ((ch ^ (r_in & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
-                                         pk[4 * ch + 2], pk[4 * ch + 3]);
-                        fence_proxy_async_smem();
-                        mbar_arrive(&stg_full[i]);
-                        if (issuer) {
-                            ok = wait_or_abort(&stg_full[i], stg_count & 1, a.err, abort_flag);
-                            if (ok) {
+                            st_shared_v4(row_addr + h * kBoxBytes + ((ch ^ (r_in & 7)) << 4), pk[h][4 * ch],
+                                         pk[h][4 * ch + 1], pk[h][4 * ch + 2], pk[h][4 * ch + 3]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&stg_full[i]);
+                    if (issuer) {
+                        ok = wait_or_abort(&stg_full[i], stg_count & 1, a.err, abort_flag);
+                        if (ok) {
+#pragma unroll
+                            for (int h = 0; h < D / 64; ++h) {
                                 if (PAGED)
-                                    tma_store_2d(&tmO, smem + C::kStageOff + i * kBoxBytes, x.head * D + 64 * h,
+                                    tma_store_2d(&tmO, smem + C::kStageOff + h * kBoxBytes, x.head * D + 64 * h,
                                                  x.qtok0 + tile_row0);
                                 else
-                                    tma_store_3d(&tmO, smem + C::kStageOff + i * kBoxBytes, 64 * h, tile_row0, x.head);
-                                bulk_commit();
-                                bulk_wait_read_all();
-                                mbar_arrive(&stg_free[i]);
+                                    tma_store_3d(&tmO, smem + C::kStageOff + h * kBoxBytes, 64 * h, tile_row0,
+                                                 x.head);
                             }
+                            bulk_commit();
+                            bulk_wait_read_all();
+                            mbar_arrive(&stg_free[0]);
                         }
-                        ++stg_count;
                     }
+                    ++stg_count;
                     if (!ok) break;
                 } else {
                     // a paged tile that ends inside the sequence's rows: plain
