@@ -10,8 +10,10 @@
 // FlashAttention-2 与 PagedAttention 实现解析" section 2.2 (block table lookup).
 //
 // Both are pure data movement (HBM-bound): 16-byte vector loads and stores,
-// one CTA per token (append) or per (block, K|V) (copy).  Out-of-range ids are
-// skipped on the device and reported through err_flag, never dereferenced.
+// one CTA per token (append); the copy runs grid-stride over 16 KiB chunks of
+// (pair, K|V) so the last wave is a fraction of a chunk, not of a block.
+// Out-of-range ids are skipped on the device and reported through err_flag,
+// never dereferenced.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -69,33 +71,44 @@ struct CopyArgs {
     uint8_t *k_cache, *v_cache;
     const int32_t *src, *dst;
     int32_t *err;
-    int num_blocks;
+    int num_blocks, num_pairs;
     long long block_bytes;  // H * block_size * d * element size (a multiple of 16)
+    int chunks;             // 16 KiB chunks per block (the last one may be short)
 };
 
-// blockIdx.x: pair, blockIdx.y: 0 = K, 1 = V.  Each thread moves 4 x 16 bytes
-// per round so several loads are in flight before the first store.
-__global__ void __launch_bounds__(512) block_copy_kernel(CopyArgs a) {
-    const int i = blockIdx.x;
-    const int s = a.src[i], d = a.dst[i];
-    if (s < 0 || s >= a.num_blocks || d < 0 || d >= a.num_blocks) {
-        if (threadIdx.x == 0 && blockIdx.y == 0 && a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
-        return;
+constexpr int kCopyThreads = 256;
+constexpr int kChunkBytes = kCopyThreads * 4 * 16;  // 4 x 16 bytes in flight per thread
+
+// Work unit w: pair w / (2 chunks), K (0) or V (1), chunk; each thread moves
+// 4 x 16 bytes with all four loads issued before the first store.
+__global__ void __launch_bounds__(kCopyThreads) block_copy_kernel(CopyArgs a) {
+    const long long units = (long long)a.num_pairs * 2 * a.chunks;
+    for (long long w = blockIdx.x; w < units; w += gridDim.x) {
+        const int i = (int)(w / (2 * a.chunks));
+        const int rem = (int)(w - (long long)i * 2 * a.chunks);
+        const int which = rem / a.chunks, c = rem - which * a.chunks;
+        const int s = a.src[i], d = a.dst[i];
+        if (s < 0 || s >= a.num_blocks || d < 0 || d >= a.num_blocks) {
+            if (threadIdx.x == 0 && which == 0 && c == 0 && a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+            continue;
+        }
+        uint8_t *base = which ? a.v_cache : a.k_cache;
+        const long long off = (long long)c * kChunkBytes;
+        const long long n = min((long long)kChunkBytes, a.block_bytes - off) / 16;  // 16-byte words of the chunk
+        const uint4 *from = reinterpret_cast<const uint4 *>(base + (size_t)s * a.block_bytes + off);
+        uint4 *to = reinterpret_cast<uint4 *>(base + (size_t)d * a.block_bytes + off);
+        const int t = threadIdx.x;
+        if (n == kChunkBytes / 16) {
+            const uint4 x0 = from[t], x1 = from[t + kCopyThreads], x2 = from[t + 2 * kCopyThreads],
+                        x3 = from[t + 3 * kCopyThreads];
+            to[t] = x0;
+            to[t + kCopyThreads] = x1;
+            to[t + 2 * kCopyThreads] = x2;
+            to[t + 3 * kCopyThreads] = x3;
+        } else {
+            for (long long k = t; k < n; k += kCopyThreads) to[k] = from[k];
+        }
     }
-    uint8_t *base = blockIdx.y ? a.v_cache : a.k_cache;
-    const uint4 *from = reinterpret_cast<const uint4 *>(base + (size_t)s * a.block_bytes);
-    uint4 *to = reinterpret_cast<uint4 *>(base + (size_t)d * a.block_bytes);
-    const long long n = a.block_bytes / 16;
-    const int stride = blockDim.x;
-    long long k = threadIdx.x;
-    for (; k + 3 * stride < n; k += 4 * stride) {
-        const uint4 x0 = from[k], x1 = from[k + stride], x2 = from[k + 2 * stride], x3 = from[k + 3 * stride];
-        to[k] = x0;
-        to[k + stride] = x1;
-        to[k + 2 * stride] = x2;
-        to[k + 3 * stride] = x3;
-    }
-    for (; k < n; k += stride) to[k] = from[k];
 }
 
 }  // namespace
@@ -129,7 +142,19 @@ attn_status launch_block_copy(const CopyLaunch &p, cudaStream_t stream) {
     a.err = p.err_flag;
     a.num_blocks = p.num_blocks;
     a.block_bytes = (long long)p.H * p.block_size * p.d * p.elem_bytes;
-    block_copy_kernel<<<dim3(p.num_pairs, 2), 512, 0, stream>>>(a);
+    a.num_pairs = p.num_pairs;
+    a.chunks = (int)((a.block_bytes + kChunkBytes - 1) / kChunkBytes);
+    static int sm_count[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ECUDA;
+    if (sm_count[dev] == 0 &&
+        cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_ECUDA;
+    const long long units = (long long)p.num_pairs * 2 * a.chunks;
+    const long long slots = 8LL * sm_count[dev];  // 8 resident 256-thread CTAs per SM
+    const int grid = (int)(units < slots ? units : slots);
+    if (grid == 0) return ATTN_OK;
+    block_copy_kernel<<<grid, kCopyThreads, 0, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
