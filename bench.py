@@ -56,6 +56,8 @@ import workloads as W  # noqa: E402
 METRIC = "prefill attn TFLOP/s & paged-decode KV GB/s, as % of B200 roofline"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures, reported beside the measured-peak fractions
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 # ---------------------------------------------------------------- helpers
@@ -910,6 +912,8 @@ def roofline(wl, per_ms, pk, pk_src, bound, clocks=None):
         peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         unit = "GB/s"
         extra = {"peak_kind": "copy bandwidth"}
+    spec = SPEC_PEAKS["bf16_tflops"] * getattr(wl, "peak_factor", 1.0) if bound == "tensor" else SPEC_PEAKS["hbm_gbs"]
+    extra["frac_of_spec"] = round(achieved / spec, 4)
     tr = recorded_traffic(wl.kernel, wl.name)
     return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": tr, "peak_source": pk_src,
