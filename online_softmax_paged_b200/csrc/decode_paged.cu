@@ -271,7 +271,6 @@ __device__ __forceinline__ void finish_item(const DecodeArgs &a, int s, int hq, 
     const int nsplit = a.item_start[s + 1] - a.item_start[s];  // (L2-resident, once per item)
     const size_t sh = (size_t)s * a.H + hq;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    (void)half;
     if (nsplit == 1) {
         if (saw_bad)
             final_store(a, sh, li, half, lane, nullptr, 0.f, -INFINITY);
