@@ -158,3 +158,15 @@ def test_fp8_rejects_other_head_dims():
     x = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(osp.AttnError):
         osp.attn_quantize_fp8(x)
+
+
+def test_fp8_many_units_per_cta_ragged():
+    """FP8 with B=2 H=90 N=300 (360 units over at most 148 CTAs, empty upper
+    tiles included) against the oracle on the dequantised operands."""
+    osp = _osp()
+    _, dev, ref = _fp8_inputs(2, 90, 300, seed=22, rotate=True)
+    O, LSE = osp.attn_fwd_fp8(dev["q8"], dev["q_scale"], dev["k8"], dev["k_scale"], dev["V"], causal=True,
+                              scale=ref["scale"])
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention_dense(ref["Q"], ref["K"], ref["V"], True, ref["scale"])
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, "fp8 many units")

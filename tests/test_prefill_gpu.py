@@ -193,3 +193,16 @@ def test_fp32_is_not_tf32():
     O, LSE = _run(inp)
     O_ref, L_ref = _full_oracle(inp)
     assert np.abs(to64(O) - O_ref).max() <= 1e-4
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_many_units_per_cta_ragged(causal):
+    """B=2 H=100 N=300: 400 units over at most 148 CTAs, so each CTA walks
+    two or three units, and every second unit's upper query tile has no rows
+    (it is skipped by the producer, the MMA issuer and the O staging order)."""
+    inp = W.dense_inputs(2, 100, 300, 128, dtype=torch.bfloat16, seed=21, device="cuda", causal=causal)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _run(inp, err)
+    assert int(err.item()) == 0
+    O_ref, L_ref = oracle.attention_dense(to64(inp["Q"]), to64(inp["K"]), to64(inp["V"]), causal, inp["scale"])
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"many units causal={causal}")
