@@ -101,9 +101,11 @@ ATTN_API size_t paged_attn_decode_workspace_size(int num_seqs, int H, int d, int
 /*
  * Bytes of device workspace paged_attn_decode_gqa needs (H_q query heads over
  * H_kv key/value heads).  Returns 0 for invalid sizes (H_q not a multiple of
- * H_kv, or as paged_attn_decode_workspace_size).  The partials are per query
- * head, so it currently equals paged_attn_decode_workspace_size(num_seqs,
- * H_q, ...); callers of paged_attn_decode_gqa should size with this one.
+ * H_kv, or as paged_attn_decode_workspace_size).  At least
+ * paged_attn_decode_workspace_size(num_seqs, H_q, ...): groups of 4 and more
+ * also need room for the partial rows of their balanced schedule (at most
+ * 1480 x 8 + num_seqs x H_q rows of d + 1 floats), which is more for few
+ * short sequences.  Callers of paged_attn_decode_gqa size with this one.
  */
 ATTN_API size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int H_q, int H_kv, int d,
                                                      int max_blocks_per_seq, int block_size);
@@ -140,8 +142,9 @@ ATTN_API int paged_attn_decode_split_tokens(int num_seqs, int H, int d, int max_
  *                0 and its LSE as -inf, and no out-of-range address is read.
  * seq_len == 0 : O = 0, LSE = -inf (no error).
  * Determinism  : the split plan and every reduction order depend only on the
- *                logical token positions, so moving blocks to other physical
- *                ids (with a matching table) gives bit-identical results.
+ *                sizes and the sequence lengths, never on the physical block
+ *                ids, so moving blocks to other physical ids (with a matching
+ *                table) gives bit-identical results.
  */
 ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache,
                               const int32_t *block_table, const int32_t *seq_lens, int block_size,
@@ -166,6 +169,15 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
  *                L2 after the first); otherwise as paged_attn_decode
  *                (whose behaviour, checks and determinism apply unchanged;
  *                paged_attn_decode is this call with H_kv = H_q).
+ * Schedule     : groups of 4 and more cut the (sequence, key/value head)
+ *                rows, laid end to end, into equal runs of 16-token tiles,
+ *                one per worker (1480 workers, runs of at least 128 tokens),
+ *                so a call's split plan depends on every sequence's length.
+ *                Groups above 8 return ATTN_EUNSUPPORTED when
+ *                num_blocks * H_kv * block_size exceeds 2^31 - 1 rows or
+ *                num_seqs * ceil(max_blocks_per_seq * block_size / 16)
+ *                exceeds 2^30 - 1 (groups of 4 and 8 then run the
+ *                split-KV kernel instead).
  */
 ATTN_API attn_status paged_attn_decode_gqa(const void *q, const void *k_cache, const void *v_cache,
                                            const int32_t *block_table, const int32_t *seq_lens, int block_size,

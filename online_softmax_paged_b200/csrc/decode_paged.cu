@@ -519,17 +519,30 @@ __global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(D
 // ------------------------------------------------------------------ grouped heads on tensor cores
 //
 // For G >= 4 query heads per key/value head the per-row shuffle reductions
-// above bound the kernel, not HBM.  This variant keeps the same item stream
-// (one warp per (sequence, split, key/value head) item, a 2-slot ring, the
-// same split-KV merge) but computes each 16-key tile with warp-level tensor
-// core MMAs (m16n8k16, bf16 in, fp32 accumulate): S = Q K^T with the G query
-// rows padded to 16, then O^T += V^T P^T, where the query heads are the
-// product's 8 columns (no padding for G = 8) and P^T's fragments are exactly
-// the S accumulators a lane holds.  K/V tiles arrive by TMA in
-// 128-byte-swizzled boxes so that the ldmatrix fragment loads are
-// conflict-free.
+// above bound the kernel, not HBM.  This variant computes each 16-key tile
+// with warp-level tensor core MMAs (m16n8k16, bf16 in, fp32 accumulate):
+// S = Q K^T with the G query rows padded to 16, then O^T += V^T P^T, where
+// the query heads are the product's 8 columns (no padding for G = 8) and
+// P^T's fragments are exactly the S accumulators a lane holds.  K/V tiles
+// arrive by TMA in 128-byte-swizzled boxes so that the ldmatrix fragment
+// loads are conflict-free.
+//
+// Work is not taken from a queue: every (sequence, key/value head) row has
+// ceil(L / 16) tiles, the rows are laid end to end (sequence-major), and
+// worker w of kWorkers takes tiles [w c, (w + 1) c) of that line, with
+// c = max(ceil(T / kWorkers), kMinTiles) for T tiles in all.  Every worker
+// then streams the same number of bytes (the last one fewer), whatever the
+// length mix; a worker's run crosses row boundaries as it comes.  A row cut
+// by worker boundaries into n segments gets n partials, stored at slots
+// worker + row (so one row's slots are consecutive, and all slots fit in
+// kWorkers + rows), and is merged by the worker that completes its last
+// segment.  The plan depends on the lengths and sizes only (kWorkers is a
+// constant, not the GPU's warp count), so results do not depend on the
+// physical block ids or on which warp ran a worker.
 
 constexpr int kMmaWarps = 10;
+constexpr int kWorkers = 1480;  // schedule width (148 SMs x 10 warps)
+constexpr int kMinTiles = 8;    // shortest worker run: 128 keys
 constexpr int kScratchBytes = 8 * kD * 4;  // per warp: up to 8 unnormalised O rows (fp32)
 constexpr int kMmaSmem = kMmaWarps * (kStages * kSlotBytes + kScratchBytes) + kMmaWarps * kStages * 8 +
                          (kMaxSmemSeqs + 1) * 4 + 64 + 1024;
@@ -568,9 +581,92 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
     return (uint32_t)((c >> 3) * 2048 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// One piece of a worker's run: tiles of one row (sequence s, key/value head
+// h), at most 64 cache blocks (their ids in tbl0 / tbl1, as in Item), the
+// whole of it inside one segment (the part of the row in one worker's run).
+struct SegItem {
+    int s, h, tok0, tok1, nt;  // tokens [tok0, tok1), nt 16-token tiles (0: none)
+    int lb0;                   // logical block of tok0
+    int tbl0, tbl1;
+    int slot, slot0, nsplit;   // this segment's partial slot, the row's first slot, segments of the row
+    bool first, last;          // the item opens / closes its segment
+};
+
+// Where a worker's fetch stands: worker w, its run [x, x_end) still to hand out.
+struct SchedPos {
+    int w;
+    long long x, x_begin, x_end;
+};
+
+// The next item of this warp (all lanes): the rest of the current worker's
+// run, then the next worker (w + warps in the grid), until none is left.
+__device__ __forceinline__ void next_seg_item(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
+                                              long long nw, int stride, int lane, int &s_hint, SchedPos &ps,
+                                              SegItem &it) {
+    if (ps.x >= ps.x_end) {
+        ps.w += stride;
+        if (ps.w >= nw) {
+            it.nt = 0;
+            return;
+        }
+        ps.x_begin = ps.x = (long long)ps.w * chunk;
+        ps.x_end = min(T, ps.x + chunk);
+    }
+    // the sequence whose rows hold tile x: Hkv starts[s] <= x < Hkv starts[s + 1]
+    const int c = (int)(ps.x / a.Hkv);
+    int lo = 0, hi = a.num_seqs - 1;
+    if (starts[s_hint] <= c && c < starts[s_hint + 1]) {
+        lo = s_hint;
+    } else {
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (starts[mid] <= c) lo = mid; else hi = mid - 1;
+        }
+    }
+    s_hint = lo;
+    const int nts = starts[lo + 1] - starts[lo];
+    const long long rb = (long long)a.Hkv * starts[lo];
+    const int h = (int)((ps.x - rb) / nts);
+    const long long row_begin = rb + (long long)h * nts, row_end = row_begin + nts;
+    const int t = (int)(ps.x - row_begin);
+    const long long seg_end = min(row_end, ps.x_end);
+    const int L = a.seq_lens[lo];
+    const int tok0 = t * kTileTok;
+    const int lb0 = tok0 / a.block_size;
+    const int tcap = (lb0 + 64) * (a.block_size / kTileTok);  // tiles of the 64 blocks from lb0
+    const int t1 = (int)min((long long)tcap, (long long)t + (seg_end - ps.x));
+    it.s = lo;
+    it.h = h;
+    it.tok0 = tok0;
+    it.tok1 = min(L, t1 * kTileTok);
+    it.nt = t1 - t;
+    it.lb0 = lb0;
+    it.first = ps.x == ps.x_begin || t == 0;
+    it.last = ps.x + it.nt == seg_end;
+    const int r = lo * a.Hkv + h;
+    it.slot = ps.w + r;
+    it.slot0 = (int)(row_begin / chunk) + r;
+    it.nsplit = (int)((row_end - 1) / chunk - row_begin / chunk) + 1;
+    const int room = a.max_blocks - lb0;
+    const int32_t *row = a.block_table + (size_t)lo * a.max_blocks + lb0;
+    const int b0 = lane < room ? __ldg(row + lane) : -1;
+    const int b1 = lane + 32 < room ? __ldg(row + 32 + lane) : -1;
+    const int nblk = (it.tok1 - 1) / a.block_size - lb0 + 1;  // <= 64
+    it.tbl0 = lane < nblk ? b0 : -1;
+    it.tbl1 = lane + 32 < nblk ? b1 : -1;
+    ps.x += it.nt;
+}
+
+// Physical block of tile t of a schedule item (all lanes; -1 when out of range).
+__device__ __forceinline__ int seg_tile_block(const DecodeArgs &a, const SegItem &it, int t) {
+    const int bi = (it.tok0 + t * kTileTok) / a.block_size - it.lb0;
+    const int v = __shfl_sync(0xffffffffu, bi < 32 ? it.tbl0 : it.tbl1, bi & 31);
+    return (v >= 0 && v < a.num_blocks) ? v : -1;
+}
+
 // Lane 0: the TMA copies of tile t of `it` (K and V, 2 boxes each).
 __device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtensorMap *tmK, const CUtensorMap *tmV,
-                                               uint8_t *slots, uint64_t *full, int slot, const Item &it, int t,
+                                               uint8_t *slots, uint64_t *full, int slot, const SegItem &it, int t,
                                                int phys) {
     uint64_t *bar = full + slot;
     if (phys < 0) {
@@ -589,52 +685,112 @@ __device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtens
     tma_load_2d(dst + kTileBytes + 2048, tmV, bar, 64, y);
 }
 
-// The final rows of query heads sh0 .. sh0 + G - 1 of sequence s (those set
-// in `mask`) from their nsplit partials: every row's loads of split q go out
-// together, so the G rows share the latency of one (the same per-row
-// arithmetic order as merge_row).
+// The final rows of query heads sh0 .. sh0 + G - 1 of sequence s from the
+// nsplit partials in slots slot0 .. slot0 + nsplit - 1 (slot q holds G rows:
+// log2-sum-exps at part_lse[q G + g], normalised rows at part_o[(q G + g) d]).
+// Up to kScratchBytes / (4 G) partials: lane j reads the log2-sum-exps of
+// partials j, j + 32, ... (one round trip per 32), the row maxima and weight
+// sums are warp reductions, the weights go to `wbuf` (the warp's scratch,
+// free once the partial is out) and the rows are read 32 / G partials at a
+// time, so 32 loads per lane are in flight together.  More partials: the
+// same sums, one partial after another.  Either way the order of every sum
+// depends only on the partial's index.
 template <int G>
-__device__ __forceinline__ void merge_rows(const DecodeArgs &a, int s, size_t sh0, int nsplit, int lane,
-                                           uint32_t mask) {
+__device__ __forceinline__ void merge_rows(const DecodeArgs &a, int s, size_t sh0, int slot0, int nsplit, int lane,
+                                           float *wbuf) {
     if (__ldcg(a.seq_bad + s)) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-            if (mask >> g & 1u) {
-                *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) = make_uint2(0u, 0u);
-                if (lane == 0) a.LSE[sh0 + g] = -INFINITY;
-            }
+        for (int g = 0; g < G; ++g) {
+            *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) = make_uint2(0u, 0u);
+            if (lane == 0) a.LSE[sh0 + g] = -INFINITY;
+        }
         return;
     }
+    constexpr int kQCap = kScratchBytes / 4 / G;  // partials whose weights fit in wbuf
+    constexpr int kU = 32 / G;                    // partials per batch of row loads
+    const float *plse = a.part_lse + (size_t)slot0 * G;
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (size_t)slot0 * G * kD) + lane;
     float M[G], tot[G];
     float4 acc[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) M[g] = -INFINITY;
-#pragma unroll 2
-    for (int q = 0; q < nsplit; ++q)
-#pragma unroll
-        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(a.part_lse + (sh0 + g) * a.max_splits + q));
-#pragma unroll
     for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
         tot[g] = 0.f;
         acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-#pragma unroll 2
-    for (int q = 0; q < nsplit; ++q) {
+    if (nsplit <= kQCap) {
+        for (int q = lane; q < nsplit; q += 32)
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const size_t pidx = (sh0 + g) * a.max_splits + q;
-            const float w = ex2_approx(__ldcg(a.part_lse + pidx) - M[g]);
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + pidx * kD) + lane);
-            tot[g] += w;
-            acc[g].x = fmaf(w, v.x, acc[g].x);
-            acc[g].y = fmaf(w, v.y, acc[g].y);
-            acc[g].z = fmaf(w, v.z, acc[g].z);
-            acc[g].w = fmaf(w, v.w, acc[g].w);
+            for (int g = 0; g < G; ++g) {
+                const float x = __ldcg(plse + q * G + g);
+                wbuf[q * G + g] = x;
+                M[g] = fmaxf(M[g], x);
+            }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M[g] = fmaxf(M[g], __shfl_xor_sync(0xffffffffu, M[g], o));
+        for (int q = lane; q < nsplit; q += 32)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float w = ex2_approx(wbuf[q * G + g] - M[g]);
+                wbuf[q * G + g] = w;
+                tot[g] += w;
+            }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tot[g] += __shfl_xor_sync(0xffffffffu, tot[g], o);
+        __syncwarp();  // every weight is in wbuf
+        int q = 0;
+        for (; q + kU <= nsplit; q += kU) {
+            float4 v[kU][G];
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+#pragma unroll
+                for (int g = 0; g < G; ++g) v[u][g] = __ldcg(po + ((q + u) * G + g) * (kD / 4));
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float w = wbuf[(q + u) * G + g];
+                    acc[g].x = fmaf(w, v[u][g].x, acc[g].x);
+                    acc[g].y = fmaf(w, v[u][g].y, acc[g].y);
+                    acc[g].z = fmaf(w, v[u][g].z, acc[g].z);
+                    acc[g].w = fmaf(w, v[u][g].w, acc[g].w);
+                }
+        }
+        for (; q < nsplit; ++q)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float w = wbuf[q * G + g];
+                const float4 v = __ldcg(po + (q * G + g) * (kD / 4));
+                acc[g].x = fmaf(w, v.x, acc[g].x);
+                acc[g].y = fmaf(w, v.y, acc[g].y);
+                acc[g].z = fmaf(w, v.z, acc[g].z);
+                acc[g].w = fmaf(w, v.w, acc[g].w);
+            }
+    } else {
+#pragma unroll 2
+        for (int q = 0; q < nsplit; ++q)
+#pragma unroll
+            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(plse + q * G + g));
+#pragma unroll 2
+        for (int q = 0; q < nsplit; ++q) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float w = ex2_approx(__ldcg(plse + q * G + g) - M[g]);
+                const float4 v = __ldcg(po + (q * G + g) * (kD / 4));
+                tot[g] += w;
+                acc[g].x = fmaf(w, v.x, acc[g].x);
+                acc[g].y = fmaf(w, v.y, acc[g].y);
+                acc[g].z = fmaf(w, v.z, acc[g].z);
+                acc[g].w = fmaf(w, v.w, acc[g].w);
+            }
         }
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        if (!(mask >> g & 1u)) continue;
         const float inv = tot[g] > 0.f ? 1.f / tot[g] : 0.f;
         *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) =
             make_uint2(pack_bf16x2(acc[g].x * inv, acc[g].y * inv), pack_bf16x2(acc[g].z * inv, acc[g].w * inv));
@@ -642,53 +798,48 @@ __device__ __forceinline__ void merge_rows(const DecodeArgs &a, int s, size_t sh
     }
 }
 
-// Output of a finished grouped item: G unnormalised rows in `scratch`
-// ([G][d] fp32), row g's max / sum in lane 4g.  One fence and G parallel
-// completion counts for the whole group; rows whose last split this was are
-// merged.
+// Output of a finished segment: G unnormalised rows in `scratch` ([G][d]
+// fp32), row g's max / sum in lane 4g.  A row in one segment is written
+// directly; otherwise the partial goes to its slot, and one fence and one
+// completion count (per key/value row) later the worker that completes the
+// row's last segment merges it (with `scratch` reused for the weights).
 template <int G>
-__device__ __forceinline__ void finish_group(const DecodeArgs &a, int s, int h, int p, int lane,
-                                             const float *scratch, float m, float l, bool saw_bad) {
-    const int nsplit = a.item_start[s + 1] - a.item_start[s];
+__device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &it, int lane, float *scratch, float m,
+                                           float l, bool saw_bad) {
+    const int s = it.s;
+    const size_t sh0 = (size_t)s * a.H + (size_t)it.h * G;
     const int gl = lane & 7;  // lanes 0..G-1: the row they report
     const float mg_l = __shfl_sync(0xffffffffu, m, 4 * gl);
     const float lg_l = __shfl_sync(0xffffffffu, l, 4 * gl);
-    if (nsplit == 1) {
+    if (it.nsplit == 1) {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
-            const size_t sh = (size_t)s * a.H + h * G + g;
             const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
             const float inv = (!saw_bad && lg > 0.f) ? 1.f / lg : 0.f;
             const float4 v = *reinterpret_cast<const float4 *>(scratch + g * kD + 4 * lane);
-            *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) =
+            *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) =
                 make_uint2(pack_bf16x2(v.x * inv, v.y * inv), pack_bf16x2(v.z * inv, v.w * inv));
         }
-        if (lane < G)
-            a.LSE[(size_t)s * a.H + h * G + lane] =
-                (!saw_bad && lg_l > 0.f) ? (mg_l + __log2f(lg_l)) * kLn2 : -INFINITY;
+        if (lane < G) a.LSE[sh0 + lane] = (!saw_bad && lg_l > 0.f) ? (mg_l + __log2f(lg_l)) * kLn2 : -INFINITY;
         return;
     }
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
-        const size_t pidx = ((size_t)s * a.H + h * G + g) * a.max_splits + p;
         const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
         const float inv = lg > 0.f ? 1.f / lg : 0.f;
         const float4 v = *reinterpret_cast<const float4 *>(scratch + g * kD + 4 * lane);
-        *reinterpret_cast<float4 *>(a.part_o + pidx * kD + 4 * lane) =
+        *reinterpret_cast<float4 *>(a.part_o + ((size_t)it.slot * G + g) * kD + 4 * lane) =
             make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
     }
-    if (lane < G)
-        a.part_lse[((size_t)s * a.H + h * G + lane) * a.max_splits + p] =
-            lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
+    if (lane < G) a.part_lse[(size_t)it.slot * G + lane] = lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
     if (lane == 0 && saw_bad) atomicOr(a.seq_bad + s, 1);
-    __threadfence();  // partials (and the bad mark) before the completion counts
+    __threadfence();  // partials (and the bad mark) before the completion count
     __syncwarp();
-    bool last = false;
-    if (lane < G) last = atomicAdd(a.done_cnt + (size_t)s * a.H + h * G + lane, 1) == nsplit - 1;
-    const uint32_t lastm = __ballot_sync(0xffffffffu, last);
-    if (!lastm) return;
+    int last = 0;
+    if (lane == 0) last = atomicAdd(a.done_cnt + (size_t)s * a.Hkv + it.h, 1) == it.nsplit - 1;
+    if (!__shfl_sync(0xffffffffu, last, 0)) return;
     __threadfence();
-    merge_rows<G>(a, s, (size_t)s * a.H + h * G, nsplit, lane, lastm);
+    merge_rows<G>(a, s, sh0, it.slot0, it.nsplit, lane, scratch);
 }
 
 template <int G>
@@ -712,7 +863,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
     }
     __syncwarp();
     pdl_wait();
-    const int32_t *starts = a.item_start;
+    const int32_t *starts = a.item_start;  // tiles before each sequence
     if (a.num_seqs <= kMaxSmemSeqs) {
         int32_t *st = reinterpret_cast<int32_t *>(smem + kMmaWarps * (kStages * kSlotBytes + kScratchBytes) +
                                                   kMmaWarps * kStages * 8);
@@ -720,11 +871,18 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         __syncthreads();
         starts = st;
     }
-    const int total = starts[a.num_seqs] * a.Hkv;
+    // the schedule: T tiles in all, runs of `chunk` tiles, nw workers with work
+    const long long T = (long long)starts[a.num_seqs] * a.Hkv;
+    const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
+    const long long nw = (T + chunk - 1) / chunk;
+    const int stride = gridDim.x * kMmaWarps;
+    SchedPos ps;
+    ps.w = blockIdx.x * kMmaWarps + wid - stride;
+    ps.x = ps.x_begin = ps.x_end = 0;
     int s_hint = 0;
 
-    Item cur, nxt;
-    fetch_item<G>(a, starts, total, lane, s_hint, cur);
+    SegItem cur, nxt;
+    next_seg_item(a, starts, T, chunk, nw, stride, lane, s_hint, ps, cur);
     bool have_nxt = false, exhausted = (cur.nt == 0);
     int pq = 0, pt = 0;
     uint32_t gi = 0, gc = 0;
@@ -734,7 +892,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         for (;;) {
             const int pnt = pq ? nxt.nt : cur.nt;
             if (pt < pnt) {
-                const int phys = pq ? tile_block(a, nxt, pt) : tile_block(a, cur, pt);
+                const int phys = pq ? seg_tile_block(a, nxt, pt) : seg_tile_block(a, cur, pt);
                 if (lane == 0) issue_tile_tma(a, &tmK, &tmV, slots, full, gi % kStages, pq ? nxt : cur, pt, phys);
                 __syncwarp();
                 ++pt;
@@ -742,7 +900,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                 return true;
             }
             if (pq == 1 || exhausted) return false;
-            fetch_item<G>(a, starts, total, lane, s_hint, nxt);
+            next_seg_item(a, starts, T, chunk, nw, stride, lane, s_hint, ps, nxt);
             if (nxt.nt == 0) {
                 exhausted = true;
                 return false;
@@ -758,11 +916,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
         }
     }
     const uint32_t slots_u32 = smem_u32(slots);
+    // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
+    // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
+    uint32_t qa0[8], qa2[8];
+    float m = -INFINITY, l = 0.f;  // row gq: running max (log2 units) and this lane's part of the sum
+    // O^T accumulators: o[mb] holds dims 16mb + gq (0, 1) and 16mb + gq + 8
+    // (2, 3) of query heads 2tq (0, 2) and 2tq + 1 (1, 3)
+    float o[8][4];
+    bool saw_bad = false;
     while (cur.nt > 0) {
-        // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
-        // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
-        uint32_t qa0[8], qa2[8];
-        {
+        if (cur.first) {
             const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
                 a.q + ((size_t)cur.s * a.H + cur.h * G + (gq < G ? gq : 0)) * kD);
 #pragma unroll
@@ -770,14 +933,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                 qa0[ks] = gq < G ? __ldg(qrow + 8 * ks + tq) : 0u;
                 qa2[ks] = gq < G ? __ldg(qrow + 8 * ks + 4 + tq) : 0u;
             }
-        }
-        float m = -INFINITY, l = 0.f;  // row gq: running max (log2 units) and this lane's part of the sum
-        // O^T accumulators: o[mb] holds dims 16mb + gq (0, 1) and 16mb + gq + 8
-        // (2, 3) of query heads 2tq (0, 2) and 2tq + 1 (1, 3)
-        float o[8][4];
+            m = -INFINITY;
+            l = 0.f;
 #pragma unroll
-        for (int mb = 0; mb < 8; ++mb) o[mb][0] = o[mb][1] = o[mb][2] = o[mb][3] = 0.f;
-        bool saw_bad = false;
+            for (int mb = 0; mb < 8; ++mb) o[mb][0] = o[mb][1] = o[mb][2] = o[mb][3] = 0.f;
+            saw_bad = false;
+        }
         for (int t = 0; t < cur.nt; ++t) {
             const int slot = gc % kStages;
             if (!mbar_wait(full + slot, (gc / kStages) & 1u, a.err)) {
@@ -785,7 +946,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                 break;
             }
             const int tok = cur.tok0 + t * kTileTok;
-            const bool tile_ok = tile_block(a, cur, t) >= 0;
+            const bool tile_ok = seg_tile_block(a, cur, t) >= 0;
             saw_bad |= !tile_ok;
             if (tile_ok) {
                 const uint32_t kt = slots_u32 + slot * kSlotBytes, vt = kt + kTileBytes;
@@ -860,22 +1021,24 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
             if (gi - gc < (uint32_t)kStages) produce();
         }
         if (dead) break;
-        // unnormalised O rows -> per-warp scratch, then the common finish
-        // (final row, or partial + merge by the last split)
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        if (2 * tq < G) {
+        if (cur.last) {
+            // unnormalised O rows -> per-warp scratch, then the common finish
+            // (final row, or partial + merge by the last segment)
+            float lt = l + __shfl_xor_sync(0xffffffffu, l, 1);
+            lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+            if (2 * tq < G) {
 #pragma unroll
-            for (int mb = 0; mb < 8; ++mb) {
-                scratch[(2 * tq) * kD + 16 * mb + gq] = o[mb][0];
-                scratch[(2 * tq + 1) * kD + 16 * mb + gq] = o[mb][1];
-                scratch[(2 * tq) * kD + 16 * mb + gq + 8] = o[mb][2];
-                scratch[(2 * tq + 1) * kD + 16 * mb + gq + 8] = o[mb][3];
+                for (int mb = 0; mb < 8; ++mb) {
+                    scratch[(2 * tq) * kD + 16 * mb + gq] = o[mb][0];
+                    scratch[(2 * tq + 1) * kD + 16 * mb + gq] = o[mb][1];
+                    scratch[(2 * tq) * kD + 16 * mb + gq + 8] = o[mb][2];
+                    scratch[(2 * tq + 1) * kD + 16 * mb + gq + 8] = o[mb][3];
+                }
             }
+            __syncwarp();
+            finish_seg<G>(a, cur, lane, scratch, m, lt, saw_bad);
+            __syncwarp();  // scratch reads done before the next segment writes it
         }
-        __syncwarp();
-        finish_group<G>(a, cur.s, cur.h, cur.p, lane, scratch, m, l, saw_bad);
-        __syncwarp();  // scratch reads done before the next item writes it
         if (!have_nxt) break;
         cur = nxt;
         have_nxt = false;
@@ -894,16 +1057,27 @@ struct WsLayout {
     size_t counter, item_start, done_cnt, seq_bad, part_lse, part_o, total;
 };
 
-WsLayout ws_layout(int num_seqs, int H, int max_splits) {
+// prow: partial rows (fp32 [d] each, plus a log2-sum-exp)
+WsLayout ws_layout(int num_seqs, int H, size_t prow) {
     WsLayout w;
     w.counter = 0;
     w.item_start = 256;
     w.done_cnt = align_up(w.item_start + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
     w.seq_bad = align_up(w.done_cnt + sizeof(int32_t) * (size_t)num_seqs * H, 256);
     w.part_lse = align_up(w.seq_bad + sizeof(int32_t) * (size_t)num_seqs, 256);
-    w.part_o = align_up(w.part_lse + sizeof(float) * (size_t)num_seqs * H * max_splits, 256);
-    w.total = align_up(w.part_o + sizeof(float) * (size_t)num_seqs * H * max_splits * kD, 256);
+    w.part_o = align_up(w.part_lse + sizeof(float) * prow, 256);
+    w.total = align_up(w.part_o + sizeof(float) * prow * kD, 256);
     return w;
+}
+
+// Partial rows for these sizes: [num_seqs, H, max_splits] for the split
+// kernel; groups of 4 or more may run the scheduled kernel, whose slots hold
+// at most (kWorkers + num_seqs * H / G) x G rows (G <= 8 per slot).
+size_t partial_rows(int num_seqs, int H, int Hkv, int max_splits) {
+    const size_t split_rows = (size_t)num_seqs * H * (size_t)(max_splits < 1 ? 1 : max_splits);
+    if (H / Hkv < 4) return split_rows;
+    const size_t sched_rows = (size_t)kWorkers * 8 + (size_t)num_seqs * H;
+    return split_rows > sched_rows ? split_rows : sched_rows;
 }
 
 }  // namespace
@@ -931,7 +1105,7 @@ int decode_max_splits(int num_seqs, int H, int Hkv, int d, int max_blocks, int b
 
 size_t decode_workspace_bytes(int num_seqs, int H, int Hkv, int d, int max_blocks, int block_size) {
     const int ms = decode_max_splits(num_seqs, H, Hkv, d, max_blocks, block_size);
-    return ws_layout(num_seqs, H, ms < 1 ? 1 : ms).total;
+    return ws_layout(num_seqs, H, partial_rows(num_seqs, H, Hkv, ms)).total;
 }
 
 template <int G>
@@ -969,8 +1143,6 @@ attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int 
         attr_set[dev] = true;
     }
     const long long rows = (long long)p.num_blocks * a.kv_heads * p.block_size;
-    if (rows > 0x7fffffffLL)  // TMA row coordinates are 32-bit
-        return a.kv_div > 1 ? ATTN_EUNSUPPORTED : launch_split<G>(a, dev, sms, stream);
     CUtensorMap tk, tv;
     if (!make_tensor_map_2d_bf16(&tk, p.k_cache, kD, rows, kD, kTileTok) ||
         !make_tensor_map_2d_bf16(&tv, p.v_cache, kD, rows, kD, kTileTok))
@@ -1014,11 +1186,25 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.num_blocks = p.num_blocks;
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
-    a.split_tokens = decode_split_tokens(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
-    a.max_splits = decode_max_splits(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
-    if (a.max_splits < 1) a.max_splits = 1;
+    if (G % 8 == 0 && G > 8) {
+        // larger groups (multi-query attention): each cache head serves G / 8
+        // virtual key/value heads of 8 query heads, adjacent in the schedule,
+        // so a cache head's tiles are re-read from L2
+        a.kv_div = G / 8;
+        a.Hkv = p.H / 8;
+    }
+    // the scheduled tensor-core kernel for groups of 4 and more, unless a TMA
+    // row coordinate (32-bit) or the tile count would overflow
+    const long long kv_rows = (long long)p.num_blocks * p.Hkv * p.block_size;
+    const long long max_tiles = ((long long)p.max_blocks * p.block_size + kTileTok - 1) / kTileTok;
+    const bool sched = G >= 4 && kv_rows <= 0x7fffffffLL && (long long)p.num_seqs * max_tiles <= 0x3fffffffLL;
+    if (G >= 4 && !sched && a.kv_div > 1) return ATTN_EUNSUPPORTED;
+    const int ms = decode_max_splits(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
+    // the plan's per-sequence counts: 16-token tiles for the schedule, splits otherwise
+    a.split_tokens = sched ? kTileTok : decode_split_tokens(p.num_seqs, p.H, p.Hkv, p.d, p.max_blocks, p.block_size);
+    a.max_splits = ms < 1 ? 1 : ms;
     a.scale_log2 = p.scale * 1.4426950408889634f;
-    const WsLayout w = ws_layout(p.num_seqs, p.H, a.max_splits);
+    const WsLayout w = ws_layout(p.num_seqs, p.H, partial_rows(p.num_seqs, p.H, p.Hkv, ms));
     uint8_t *ws = static_cast<uint8_t *>(p.workspace);
     a.counter = reinterpret_cast<int32_t *>(ws + w.counter);
     a.item_start = reinterpret_cast<int32_t *>(ws + w.item_start);
@@ -1029,20 +1215,13 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
 
     decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    if (sched) return G == 4 ? launch_mma<4>(a, p, dev, sm_count[dev], stream)
+                             : launch_mma<8>(a, p, dev, sm_count[dev], stream);
     switch (G) {
         case 1: return launch_split<1>(a, dev, sm_count[dev], stream);
         case 2: return launch_split<2>(a, dev, sm_count[dev], stream);
-        case 4: return launch_mma<4>(a, p, dev, sm_count[dev], stream);
-        case 8: return launch_mma<8>(a, p, dev, sm_count[dev], stream);
-    }
-    if (G % 8 == 0) {
-        // larger groups (multi-query attention): each cache head serves G / 8
-        // virtual key/value heads of 8 query heads; the items of one cache
-        // head are consecutive in the work queue, so its tiles are re-read
-        // from L2
-        a.kv_div = G / 8;
-        a.Hkv = p.H / 8;
-        return launch_mma<8>(a, p, dev, sm_count[dev], stream);
+        case 4: return launch_split<4>(a, dev, sm_count[dev], stream);
+        case 8: return launch_split<8>(a, dev, sm_count[dev], stream);
     }
     return ATTN_EUNSUPPORTED;
 }

@@ -122,10 +122,17 @@ def test_binding_refuses_cpu_tensors():
 
 
 def test_gqa_workspace_size(lib):
-    """Grouped workspace: partials are per query head, so it equals the
-    multi-head size for every valid grouping; invalid groupings give 0."""
+    """Grouped workspace: groups of 1 and 2 need the multi-head size; groups
+    of 4 and more at least that and room for the balanced schedule's partial
+    rows (1480 runs x up to 8 heads + one per query head, d + 1 floats each),
+    which dominates for few short sequences; invalid groupings give 0."""
     mha = osp.paged_attn_decode_workspace_size(64, 32, 128, 256, 16)
-    for hkv in (32, 16, 8, 4):
+    for hkv in (32, 16):
         assert osp.paged_attn_decode_gqa_workspace_size(64, 32, hkv, 128, 256, 16) == mha
+    for hkv in (8, 4, 1):
+        assert osp.paged_attn_decode_gqa_workspace_size(64, 32, hkv, 128, 256, 16) >= mha
+    small = osp.paged_attn_decode_gqa_workspace_size(1, 8, 1, 128, 4, 16)
+    assert small > osp.paged_attn_decode_workspace_size(1, 8, 128, 4, 16)
+    assert small >= (1480 * 8 + 8) * 129 * 4
     assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 3, 128, 256, 16) == 0
     assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 0, 128, 256, 16) == 0

@@ -275,3 +275,80 @@ def test_mqa_large_groups_full(Hq, Hkv, bs):
     O2, L2 = osp.paged_attn_decode_gqa(q, p2.k_cache, p2.v_cache, p2.block_table, p2.seq_lens, bs, scale=p.scale)
     torch.cuda.synchronize()
     assert torch.equal(O, O2) and torch.equal(LSE, L2)
+
+
+def _gqa(q, p, err=None):
+    O, LSE = _osp().paged_attn_decode_gqa(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.block_size,
+                                          scale=p.scale, err_flag=err)
+    torch.cuda.synchronize()
+    return O, LSE
+
+
+def _gqa_oracle(q, p, seqs=None):
+    return oracle.paged_decode(to64(q), DeviceCache(p.k_cache), DeviceCache(p.v_cache), p.block_table.cpu().numpy(),
+                               p.seq_lens.cpu().numpy(), p.block_size, p.scale, seqs=seqs)
+
+
+@pytest.mark.parametrize("Hq,bs", [(8, 16), (4, 32)])
+def test_gqa_long_row_many_segments(Hq, bs):
+    """Groups of 4 and 8 run on a balanced schedule that cuts the (sequence,
+    key/value head) rows into equal runs of tiles.  Few tiles in all give the
+    shortest run (128 keys), so a 20000-token row is cut into more than 128
+    segments (the merge's many-partials path) beside short rows; a placement
+    shuffle is bit-identical."""
+    lens = [20000, 1, 16, 17, 700]
+    p = W.paged_uniform(H=1, d=128, block_size=bs, pool=1400, len_hi=20000, seed=90 + Hq, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(91 + Hq)
+    q = torch.randn((len(lens), Hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _gqa(q, p, err)
+    assert int(err.item()) == 0
+    O_ref, L_ref = _gqa_oracle(q, p)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"long row Hq={Hq} bs={bs}")
+    p2 = W.shuffle_placement(p, seed=7)
+    O2, L2 = _gqa(q, p2)
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
+
+
+def test_gqa_odd_runs_cut_blocks():
+    """64 sequences of 0..850 tokens, 8 key/value heads, G = 4, 32-token
+    blocks: 12776 tiles give runs of 9 tiles, so runs start and end in
+    the middle of cache blocks and rows; against the oracle, and a placement
+    shuffle is bit-identical."""
+    lens = np.random.default_rng(95).integers(0, 851, 64).tolist()  # lengths fixed on the host
+    p = W.paged_uniform(H=8, d=128, block_size=32, pool=1700, len_hi=850, seed=93, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(94)
+    q = torch.randn((64, 32, 128), generator=g, device="cuda").to(torch.bfloat16)
+    tiles = int(sum(-(-int(L) // 16) for L in lens)) * 8
+    assert -(-tiles // 1480) % 2 == 1, tiles  # an odd run length
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _gqa(q, p, err)
+    assert int(err.item()) == 0
+    O_ref, L_ref = _gqa_oracle(q, p)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, "odd runs bs=32")
+    p2 = W.shuffle_placement(p, seed=8)
+    O2, L2 = _gqa(q, p2)
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_gqa_bad_block_table_entry_in_cut_row(G):
+    """A bad block id deep inside a long row that spans several runs: the
+    error bit is set, that sequence is zeroed (O = 0, LSE = -inf) for every
+    query head, the other sequences still match the oracle."""
+    osp = _osp()
+    Hkv = 32 // G
+    lens = [3000, 5000, 40, 2500]
+    p = W.paged_uniform(H=Hkv, d=128, block_size=16, pool=700, len_hi=5000, seed=95 + G, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(96 + G)
+    q = torch.randn((len(lens), 32, 128), generator=g, device="cuda").to(torch.bfloat16)
+    t = p.block_table.clone()
+    t[1, 200] = p.num_blocks + 3
+    bad = W.PagedInputs(q, p.k_cache, p.v_cache, t, p.seq_lens, p.block_size, p.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _gqa(q, bad, err)
+    assert osp.attn_read_error(err) & osp.ATTN_DEVERR_BLOCK_TABLE
+    assert (O[1] == 0).all() and torch.isneginf(LSE[1]).all()
+    good = [0, 2, 3]
+    O_ref, L_ref = _gqa_oracle(q, p, seqs=good)
+    check_close(O[good], LSE[good], O_ref[good], L_ref[good], torch.bfloat16, f"G={G} good rows beside a bad one")
