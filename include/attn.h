@@ -171,8 +171,10 @@ ATTN_API attn_status paged_attn_decode(const void *q, const void *k_cache, const
  *                paged_attn_decode is this call with H_kv = H_q).
  * Schedule     : groups of 4 and more cut the (sequence, key/value head)
  *                rows, laid end to end, into equal runs of 16-token tiles,
- *                one per worker (1480 workers, runs of at least 128 tokens),
- *                so a call's split plan depends on every sequence's length.
+ *                one per worker (1184 workers, runs of at least 128 tokens),
+ *                so a call's split plan depends on every sequence's length;
+ *                rows cut into several runs are merged by a second kernel
+ *                on the same stream.
  *                Groups above 8 return ATTN_EUNSUPPORTED when
  *                num_blocks * H_kv * block_size exceeds 2^31 - 1 rows or
  *                num_seqs * ceil(max_blocks_per_seq * block_size / 16)

@@ -82,6 +82,7 @@ struct DecodeArgs {
     int Hkv;              // key/value heads of the item space; H (query heads) = Hkv * G
     int kv_heads;         // key/value heads of the cache (= Hkv, or Hkv / kv_div)
     int kv_div;           // groups above 8 run as kv_div groups of 8 per cache head
+    int bs_shift;         // log2(block_size)
     float scale_log2;     // scale * log2(e)
 };
 
@@ -539,13 +540,28 @@ __global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(D
 // segment.  The plan depends on the lengths and sizes only (kWorkers is a
 // constant, not the GPU's warp count), so results do not depend on the
 // physical block ids or on which warp ran a worker.
+//
+// A CTA is 8 math warps and one producer warp (in a warpgroup of its own,
+// the register split moving registers to the math warps).  Lane c of the
+// producer walks math warp c's schedule tile by tile, reads the block ids
+// one tile ahead, and issues each tile's TMA copies into warp c's 2-slot ring
+// as soon as the warp releases the slot (full / empty mbarriers per slot),
+// so the math warps only wait, compute and release.
 
-constexpr int kMmaWarps = 10;
-constexpr int kWorkers = 1480;  // schedule width (148 SMs x 10 warps)
-constexpr int kMinTiles = 8;    // shortest worker run: 128 keys
-constexpr int kScratchBytes = 8 * kD * 4;  // per warp: up to 8 unnormalised O rows (fp32)
-constexpr int kMmaSmem = kMmaWarps * (kStages * kSlotBytes + kScratchBytes) + kMmaWarps * kStages * 8 +
-                         (kMaxSmemSeqs + 1) * 4 + 64 + 1024;
+constexpr int kCons = 8;                          // math warps per CTA
+constexpr int kMmaThreads = (kCons + 4) * 32;     // + the producer's warpgroup
+constexpr int kConsRegs = 224, kProdRegs = 56;    // 256 x 224 + 128 x 56 = 384 x 168
+constexpr int kWorkers = 148 * kCons;             // schedule width: one worker per math warp of 148 SMs
+constexpr int kMaxWorkers = 148 * 10;             // workspace bound (at least kWorkers)
+constexpr int kMinTiles = 8;                      // shortest worker run: 128 keys
+constexpr float kLazyLog2 = 8.f;  // rescale only when the max grows by more than 2^8
+constexpr int kScratchBytes = 8 * kD * 4;  // per math warp: up to 8 unnormalised O rows (fp32)
+constexpr int kRingBytes = kCons * kStages * kSlotBytes;
+constexpr int kBarOff = kRingBytes + kCons * kScratchBytes;    // full[kCons][2], empty[kCons][2]
+constexpr int kBadOff = kBarOff + 2 * kCons * kStages * 8;      // slot_bad[kCons][2] (int)
+constexpr int kStartsOff = kBadOff + kCons * kStages * 4;
+constexpr int kMmaSmem = kStartsOff + (kMaxSmemSeqs + 1) * 4 + 1024;
+static_assert(kConsRegs * kCons * 32 + kProdRegs * 128 <= 168 * kMmaThreads, "register split");
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -581,237 +597,145 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
     return (uint32_t)((c >> 3) * 2048 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// One piece of a worker's run: tiles of one row (sequence s, key/value head
-// h), at most 64 cache blocks (their ids in tbl0 / tbl1, as in Item), the
-// whole of it inside one segment (the part of the row in one worker's run).
+// Non-blocking probe of an mbarrier phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// One piece of a math warp's run: tiles of one row (sequence s, key/value
+// head h), the whole of it inside one segment (the part of the row in one
+// worker's run).
 struct SegItem {
     int s, h, tok0, tok1, nt;  // tokens [tok0, tok1), nt 16-token tiles (0: none)
-    int lb0;                   // logical block of tok0
-    int tbl0, tbl1;
-    int slot, slot0, nsplit;   // this segment's partial slot, the row's first slot, segments of the row
+    int w;                     // the worker whose run holds the item
     bool first, last;          // the item opens / closes its segment
 };
 
-// Where a worker's fetch stands: worker w, its run [x, x_end) still to hand out.
+// Where a worker's walk stands: worker w, its run [x, x_end) still to go.
 struct SchedPos {
     int w;
     long long x, x_begin, x_end;
 };
 
-// The next item of this warp (all lanes): the rest of the current worker's
-// run, then the next worker (w + warps in the grid), until none is left.
-__device__ __forceinline__ void next_seg_item(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
-                                              long long nw, int stride, int lane, int &s_hint, SchedPos &ps,
-                                              SegItem &it) {
-    if (ps.x >= ps.x_end) {
-        ps.w += stride;
-        if (ps.w >= nw) {
-            it.nt = 0;
-            return;
-        }
-        ps.x_begin = ps.x = (long long)ps.w * chunk;
-        ps.x_end = min(T, ps.x + chunk);
-    }
-    // the sequence whose rows hold tile x: Hkv starts[s] <= x < Hkv starts[s + 1]
-    const int c = (int)(ps.x / a.Hkv);
+// The sequence whose rows hold tile x: Hkv starts[s] <= x < Hkv starts[s + 1]
+// (starts: tiles before each sequence; empty sequences share a start).
+__device__ __forceinline__ int seq_of_tile(const DecodeArgs &a, const int32_t *starts, long long x, int s_hint) {
+    const int c = (int)(x / a.Hkv);
+    if (starts[s_hint] <= c && c < starts[s_hint + 1]) return s_hint;
     int lo = 0, hi = a.num_seqs - 1;
-    if (starts[s_hint] <= c && c < starts[s_hint + 1]) {
-        lo = s_hint;
-    } else {
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (starts[mid] <= c) lo = mid; else hi = mid - 1;
-        }
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (starts[mid] <= c) lo = mid; else hi = mid - 1;
     }
-    s_hint = lo;
-    const int nts = starts[lo + 1] - starts[lo];
-    const long long rb = (long long)a.Hkv * starts[lo];
+    return lo;
+}
+
+// Start worker run ps.w + stride (false: none left).
+__device__ __forceinline__ bool next_worker(SchedPos &ps, long long T, int chunk, long long nw, int stride) {
+    ps.w += stride;
+    if (ps.w >= nw) return false;
+    ps.x_begin = ps.x = (long long)ps.w * chunk;
+    ps.x_end = min(T, ps.x + chunk);
+    return true;
+}
+
+// The next item of a math warp (warp-uniform): the rest of the current row
+// inside the current worker's run, then the next worker (w + stride).
+__device__ __forceinline__ void next_seg_item(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
+                                              long long nw, int stride, int &s_hint, SchedPos &ps, SegItem &it) {
+    if (ps.x >= ps.x_end && !next_worker(ps, T, chunk, nw, stride)) {
+        it.nt = 0;
+        return;
+    }
+    const int s = seq_of_tile(a, starts, ps.x, s_hint);
+    s_hint = s;
+    const int nts = starts[s + 1] - starts[s];
+    const long long rb = (long long)a.Hkv * starts[s];
     const int h = (int)((ps.x - rb) / nts);
     const long long row_begin = rb + (long long)h * nts, row_end = row_begin + nts;
     const int t = (int)(ps.x - row_begin);
     const long long seg_end = min(row_end, ps.x_end);
-    const int L = a.seq_lens[lo];
-    const int tok0 = t * kTileTok;
-    const int lb0 = tok0 / a.block_size;
-    const int tcap = (lb0 + 64) * (a.block_size / kTileTok);  // tiles of the 64 blocks from lb0
-    const int t1 = (int)min((long long)tcap, (long long)t + (seg_end - ps.x));
-    it.s = lo;
+    it.s = s;
     it.h = h;
-    it.tok0 = tok0;
-    it.tok1 = min(L, t1 * kTileTok);
-    it.nt = t1 - t;
-    it.lb0 = lb0;
+    it.tok0 = t * kTileTok;
+    it.nt = (int)(seg_end - ps.x);
+    it.tok1 = min(a.seq_lens[s], (t + it.nt) * kTileTok);
+    it.w = ps.w;
     it.first = ps.x == ps.x_begin || t == 0;
-    it.last = ps.x + it.nt == seg_end;
-    const int r = lo * a.Hkv + h;
-    it.slot = ps.w + r;
-    it.slot0 = (int)(row_begin / chunk) + r;
-    it.nsplit = (int)((row_end - 1) / chunk - row_begin / chunk) + 1;
-    const int room = a.max_blocks - lb0;
-    const int32_t *row = a.block_table + (size_t)lo * a.max_blocks + lb0;
-    const int b0 = lane < room ? __ldg(row + lane) : -1;
-    const int b1 = lane + 32 < room ? __ldg(row + 32 + lane) : -1;
-    const int nblk = (it.tok1 - 1) / a.block_size - lb0 + 1;  // <= 64
-    it.tbl0 = lane < nblk ? b0 : -1;
-    it.tbl1 = lane + 32 < nblk ? b1 : -1;
-    ps.x += it.nt;
+    it.last = true;  // an item is a whole segment
+    ps.x = seg_end;
 }
 
-// Physical block of tile t of a schedule item (all lanes; -1 when out of range).
-__device__ __forceinline__ int seg_tile_block(const DecodeArgs &a, const SegItem &it, int t) {
-    const int bi = (it.tok0 + t * kTileTok) / a.block_size - it.lb0;
-    const int v = __shfl_sync(0xffffffffu, bi < 32 ? it.tbl0 : it.tbl1, bi & 31);
-    return (v >= 0 && v < a.num_blocks) ? v : -1;
+// Producer lane: the tile it issues next for its math warp, walked tile by
+// tile through the same schedule (row s, h at tile t of nts).
+struct TileWalk {
+    SchedPos ps;
+    int s, h, t, nts;
+    int id;  // block id of the tile (read one tile ahead)
+    bool live;
+};
+
+__device__ __forceinline__ void walk_locate(const DecodeArgs &a, const int32_t *starts, TileWalk &wk) {
+    wk.s = seq_of_tile(a, starts, wk.ps.x, wk.s);
+    wk.nts = starts[wk.s + 1] - starts[wk.s];
+    const long long rel = wk.ps.x - (long long)a.Hkv * starts[wk.s];
+    wk.h = (int)(rel / wk.nts);
+    wk.t = (int)(rel - (long long)wk.h * wk.nts);
 }
 
-// Lane 0: the TMA copies of tile t of `it` (K and V, 2 boxes each).
-__device__ __forceinline__ void issue_tile_tma(const DecodeArgs &a, const CUtensorMap *tmK, const CUtensorMap *tmV,
-                                               uint8_t *slots, uint64_t *full, int slot, const SegItem &it, int t,
-                                               int phys) {
-    uint64_t *bar = full + slot;
-    if (phys < 0) {
-        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
-        mbar_arrive(bar);
-        return;
-    }
-    const int tok = it.tok0 + t * kTileTok;
-    const int y = (phys * a.kv_heads + it.h / a.kv_div) * a.block_size + (tok % a.block_size);
-    uint8_t *dst = slots + slot * kSlotBytes;
-    fence_proxy_async_smem();  // the warp's generic writes to the slot (dead-row zeroing) come first
-    mbar_arrive_expect_tx(bar, kSlotBytes);
-    tma_load_2d(dst, tmK, bar, 0, y);
-    tma_load_2d(dst + 2048, tmK, bar, 64, y);
-    tma_load_2d(dst + kTileBytes, tmV, bar, 0, y);
-    tma_load_2d(dst + kTileBytes + 2048, tmV, bar, 64, y);
+__device__ __forceinline__ int walk_block_id(const DecodeArgs &a, const TileWalk &wk) {
+    return __ldg(a.block_table + (size_t)wk.s * a.max_blocks + ((wk.t * kTileTok) >> a.bs_shift));
 }
 
-// The final rows of query heads sh0 .. sh0 + G - 1 of sequence s from the
-// nsplit partials in slots slot0 .. slot0 + nsplit - 1 (slot q holds G rows:
-// log2-sum-exps at part_lse[q G + g], normalised rows at part_o[(q G + g) d]).
-// Up to kScratchBytes / (4 G) partials: lane j reads the log2-sum-exps of
-// partials j, j + 32, ... (one round trip per 32), the row maxima and weight
-// sums are warp reductions, the weights go to `wbuf` (the warp's scratch,
-// free once the partial is out) and the rows are read 32 / G partials at a
-// time, so 32 loads per lane are in flight together.  More partials: the
-// same sums, one partial after another.  Either way the order of every sum
-// depends only on the partial's index.
-template <int G>
-__device__ __forceinline__ void merge_rows(const DecodeArgs &a, int s, size_t sh0, int slot0, int nsplit, int lane,
-                                           float *wbuf) {
-    if (__ldcg(a.seq_bad + s)) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) = make_uint2(0u, 0u);
-            if (lane == 0) a.LSE[sh0 + g] = -INFINITY;
-        }
-        return;
+// Step to the next tile (false: the math warp's schedule is done).
+__device__ __forceinline__ bool walk_advance(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
+                                             long long nw, int stride, TileWalk &wk) {
+    ++wk.ps.x;
+    if (wk.ps.x >= wk.ps.x_end) {
+        if (!next_worker(wk.ps, T, chunk, nw, stride)) return false;
+        walk_locate(a, starts, wk);
+        return true;
     }
-    constexpr int kQCap = kScratchBytes / 4 / G;  // partials whose weights fit in wbuf
-    constexpr int kU = 32 / G;                    // partials per batch of row loads
-    const float *plse = a.part_lse + (size_t)slot0 * G;
-    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (size_t)slot0 * G * kD) + lane;
-    float M[G], tot[G];
-    float4 acc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        M[g] = -INFINITY;
-        tot[g] = 0.f;
-        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (nsplit <= kQCap) {
-        for (int q = lane; q < nsplit; q += 32)
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float x = __ldcg(plse + q * G + g);
-                wbuf[q * G + g] = x;
-                M[g] = fmaxf(M[g], x);
-            }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) M[g] = fmaxf(M[g], __shfl_xor_sync(0xffffffffu, M[g], o));
-        for (int q = lane; q < nsplit; q += 32)
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float w = ex2_approx(wbuf[q * G + g] - M[g]);
-                wbuf[q * G + g] = w;
-                tot[g] += w;
-            }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) tot[g] += __shfl_xor_sync(0xffffffffu, tot[g], o);
-        __syncwarp();  // every weight is in wbuf
-        int q = 0;
-        for (; q + kU <= nsplit; q += kU) {
-            float4 v[kU][G];
-#pragma unroll
-            for (int u = 0; u < kU; ++u)
-#pragma unroll
-                for (int g = 0; g < G; ++g) v[u][g] = __ldcg(po + ((q + u) * G + g) * (kD / 4));
-#pragma unroll
-            for (int u = 0; u < kU; ++u)
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float w = wbuf[(q + u) * G + g];
-                    acc[g].x = fmaf(w, v[u][g].x, acc[g].x);
-                    acc[g].y = fmaf(w, v[u][g].y, acc[g].y);
-                    acc[g].z = fmaf(w, v[u][g].z, acc[g].z);
-                    acc[g].w = fmaf(w, v[u][g].w, acc[g].w);
-                }
-        }
-        for (; q < nsplit; ++q)
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float w = wbuf[q * G + g];
-                const float4 v = __ldcg(po + (q * G + g) * (kD / 4));
-                acc[g].x = fmaf(w, v.x, acc[g].x);
-                acc[g].y = fmaf(w, v.y, acc[g].y);
-                acc[g].z = fmaf(w, v.z, acc[g].z);
-                acc[g].w = fmaf(w, v.w, acc[g].w);
-            }
-    } else {
-#pragma unroll 2
-        for (int q = 0; q < nsplit; ++q)
-#pragma unroll
-            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(plse + q * G + g));
-#pragma unroll 2
-        for (int q = 0; q < nsplit; ++q) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float w = ex2_approx(__ldcg(plse + q * G + g) - M[g]);
-                const float4 v = __ldcg(po + (q * G + g) * (kD / 4));
-                tot[g] += w;
-                acc[g].x = fmaf(w, v.x, acc[g].x);
-                acc[g].y = fmaf(w, v.y, acc[g].y);
-                acc[g].z = fmaf(w, v.z, acc[g].z);
-                acc[g].w = fmaf(w, v.w, acc[g].w);
-            }
+    if (++wk.t == wk.nts) {
+        wk.t = 0;
+        if (++wk.h == a.Hkv) {
+            wk.h = 0;
+            do {
+                ++wk.s;
+            } while (starts[wk.s + 1] == starts[wk.s]);  // tile x lies in a later, non-empty sequence
+            wk.nts = starts[wk.s + 1] - starts[wk.s];
         }
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float inv = tot[g] > 0.f ? 1.f / tot[g] : 0.f;
-        *reinterpret_cast<uint2 *>(a.O + (sh0 + g) * kD + 4 * lane) =
-            make_uint2(pack_bf16x2(acc[g].x * inv, acc[g].y * inv), pack_bf16x2(acc[g].z * inv, acc[g].w * inv));
-        if (lane == 0) a.LSE[sh0 + g] = tot[g] > 0.f ? (M[g] + __log2f(tot[g])) * kLn2 : -INFINITY;
-    }
+    return true;
 }
 
 // Output of a finished segment: G unnormalised rows in `scratch` ([G][d]
 // fp32), row g's max / sum in lane 4g.  A row in one segment is written
-// directly; otherwise the partial goes to its slot, and one fence and one
-// completion count (per key/value row) later the worker that completes the
-// row's last segment merges it (with `scratch` reused for the weights).
+// directly; otherwise the partial goes to its slot for decode_merge_kernel.
 template <int G>
-__device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &it, int lane, float *scratch, float m,
-                                           float l, bool saw_bad) {
+__device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &it, const int32_t *starts, int chunk,
+                                           int lane, float *scratch, float m, float l, bool saw_bad) {
     const int s = it.s;
+    // the row's place in the schedule: its tiles [row_begin, row_begin + nts)
+    // span workers row_begin / chunk .. (row_begin + nts - 1) / chunk
+    const int nts = starts[s + 1] - starts[s];
+    const long long row_begin = (long long)a.Hkv * starts[s] + (long long)it.h * nts;
+    const int r = s * a.Hkv + it.h;
+    const int nsplit = (int)((row_begin + nts - 1) / chunk - row_begin / chunk) + 1;
+    const int slot = it.w + r;
     const size_t sh0 = (size_t)s * a.H + (size_t)it.h * G;
     const int gl = lane & 7;  // lanes 0..G-1: the row they report
     const float mg_l = __shfl_sync(0xffffffffu, m, 4 * gl);
     const float lg_l = __shfl_sync(0xffffffffu, l, 4 * gl);
-    if (it.nsplit == 1) {
+    if (nsplit == 1) {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
             const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
@@ -828,104 +752,144 @@ __device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &i
         const float lg = __shfl_sync(0xffffffffu, l, 4 * g);
         const float inv = lg > 0.f ? 1.f / lg : 0.f;
         const float4 v = *reinterpret_cast<const float4 *>(scratch + g * kD + 4 * lane);
-        *reinterpret_cast<float4 *>(a.part_o + ((size_t)it.slot * G + g) * kD + 4 * lane) =
+        *reinterpret_cast<float4 *>(a.part_o + ((size_t)slot * G + g) * kD + 4 * lane) =
             make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
     }
-    if (lane < G) a.part_lse[(size_t)it.slot * G + lane] = lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
+    if (lane < G) a.part_lse[(size_t)slot * G + lane] = lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
     if (lane == 0 && saw_bad) atomicOr(a.seq_bad + s, 1);
-    __threadfence();  // partials (and the bad mark) before the completion count
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(a.done_cnt + (size_t)s * a.Hkv + it.h, 1) == it.nsplit - 1;
-    if (!__shfl_sync(0xffffffffu, last, 0)) return;
-    __threadfence();
-    merge_rows<G>(a, s, sh0, it.slot0, it.nsplit, lane, scratch);
 }
 
 template <int G>
-__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+__global__ void __launch_bounds__(kMmaThreads, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DecodeArgs a) {
     static_assert(G == 4 || G == 8, "query group of 4 or 8");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head of the group) and column pair
-    uint8_t *slots = smem + (size_t)wid * kStages * kSlotBytes;
-    float *scratch = reinterpret_cast<float *>(smem + kMmaWarps * kStages * kSlotBytes + wid * kScratchBytes);
-    uint64_t *full =
-        reinterpret_cast<uint64_t *>(smem + kMmaWarps * (kStages * kSlotBytes + kScratchBytes)) + wid * kStages;
-    if (lane == 0) {
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);  // [kCons][kStages]
+    uint64_t *empty = full + kCons * kStages;                       // [kCons][kStages]
+    volatile int32_t *slot_bad = reinterpret_cast<int32_t *>(smem + kBadOff);
+    if (threadIdx.x == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        for (int i = 0; i < kStages; ++i) mbar_init(full + i, 1);
+        for (int i = 0; i < kCons * kStages; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, 1);
+        }
         fence_barrier_init();
     }
-    __syncwarp();
     pdl_wait();
+    pdl_launch_dependents();  // the merge grid may be set up now; it waits for this grid's end
     const int32_t *starts = a.item_start;  // tiles before each sequence
     if (a.num_seqs <= kMaxSmemSeqs) {
-        int32_t *st = reinterpret_cast<int32_t *>(smem + kMmaWarps * (kStages * kSlotBytes + kScratchBytes) +
-                                                  kMmaWarps * kStages * 8);
+        int32_t *st = reinterpret_cast<int32_t *>(smem + kStartsOff);
         for (int i = threadIdx.x; i <= a.num_seqs; i += blockDim.x) st[i] = a.item_start[i];
-        __syncthreads();
         starts = st;
     }
+    __syncthreads();  // barriers initialised, offsets staged
     // the schedule: T tiles in all, runs of `chunk` tiles, nw workers with work
     const long long T = (long long)starts[a.num_seqs] * a.Hkv;
     const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
     const long long nw = (T + chunk - 1) / chunk;
-    const int stride = gridDim.x * kMmaWarps;
+    const int stride = gridDim.x * kCons;
+
+    if (wid >= kCons) {
+        // ---------------- producer warpgroup: warp kCons issues, the rest leave
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProdRegs));
+        if (wid != kCons) return;
+        const int c = lane;  // the math warp this lane serves
+        TileWalk wk;
+        wk.ps.w = blockIdx.x * kCons + c - stride;
+        wk.ps.x = wk.ps.x_end = 0;
+        wk.s = 0;
+        wk.live = c < kCons && next_worker(wk.ps, T, chunk, nw, stride);
+        if (wk.live) {
+            walk_locate(a, starts, wk);
+            wk.id = walk_block_id(a, wk);
+        }
+        uint32_t gi = 0;
+        uint64_t t_last = globaltimer_ns();
+        bool timed_out = false;
+        while (__any_sync(0xffffffffu, wk.live)) {
+            bool issued = false;
+            if (wk.live) {
+                const int slot = gi % kStages;
+                uint64_t *fb = full + c * kStages + slot;
+                // a non-blocking probe: one lane's wait must not hold up the others
+                if (mbar_test_wait(empty + c * kStages + slot, ((gi / kStages) & 1u) ^ 1u)) {
+                    issued = true;
+                    const int id = wk.id;
+                    if (id < 0 || id >= a.num_blocks) {
+                        // never read: the math warp skips the tile and marks the sequence
+                        slot_bad[c * kStages + slot] = 1;
+                        if (a.err) atomicOr(a.err, ATTN_DEVERR_BLOCK_TABLE);
+                        mbar_arrive(fb);
+                    } else {
+                        slot_bad[c * kStages + slot] = 0;
+                        const int y = ((id * a.kv_heads + wk.h / a.kv_div) << a.bs_shift) +
+                                      ((wk.t * kTileTok) & (a.block_size - 1));
+                        uint8_t *dst = smem + (c * kStages + slot) * kSlotBytes;
+                        mbar_arrive_expect_tx(fb, kSlotBytes);
+                        tma_load_2d(dst, &tmK, fb, 0, y);
+                        tma_load_2d(dst + 2048, &tmK, fb, 64, y);
+                        tma_load_2d(dst + kTileBytes, &tmV, fb, 0, y);
+                        tma_load_2d(dst + kTileBytes + 2048, &tmV, fb, 64, y);
+                    }
+                    ++gi;
+                    wk.live = walk_advance(a, starts, T, chunk, nw, stride, wk);
+                    if (wk.live) wk.id = walk_block_id(a, wk);  // consumed at the next issue
+                    t_last = globaltimer_ns();
+                }
+            }
+            if (!__any_sync(0xffffffffu, issued)) {
+                __nanosleep(64);  // nothing to refill: leave the issue slots to the math warps
+                // bounded: a math warp that stopped consuming (its own wait ran
+                // out) ends this loop after the wait limit
+                if (wk.live && globaltimer_ns() - t_last > kWaitLimitNs) {
+                    timed_out = true;
+                    wk.live = false;
+                }
+            }
+        }
+        if (timed_out && a.err) atomicOr(a.err, ATTN_DEVERR_TIMEOUT);
+        // copies still in flight land before the CTA may exit
+        if (c < kCons) {
+            for (uint32_t k = gi > kStages ? gi - kStages : 0; k < gi; ++k)
+                mbar_wait(full + c * kStages + k % kStages, (k / kStages) & 1u, nullptr);
+        }
+        return;
+    }
+
+    // ---------------- math warps
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsRegs));
+    const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head of the group) and column pair
+    uint8_t *slots = smem + (size_t)wid * kStages * kSlotBytes;
+    float *scratch = reinterpret_cast<float *>(smem + kRingBytes + wid * kScratchBytes);
+    uint64_t *my_full = full + wid * kStages, *my_empty = empty + wid * kStages;
     SchedPos ps;
-    ps.w = blockIdx.x * kMmaWarps + wid - stride;
+    ps.w = blockIdx.x * kCons + wid - stride;
     ps.x = ps.x_begin = ps.x_end = 0;
     int s_hint = 0;
-
-    SegItem cur, nxt;
-    next_seg_item(a, starts, T, chunk, nw, stride, lane, s_hint, ps, cur);
-    bool have_nxt = false, exhausted = (cur.nt == 0);
-    int pq = 0, pt = 0;
-    uint32_t gi = 0, gc = 0;
-    bool dead = false;
-
-    auto produce = [&]() -> bool {
-        for (;;) {
-            const int pnt = pq ? nxt.nt : cur.nt;
-            if (pt < pnt) {
-                const int phys = pq ? seg_tile_block(a, nxt, pt) : seg_tile_block(a, cur, pt);
-                if (lane == 0) issue_tile_tma(a, &tmK, &tmV, slots, full, gi % kStages, pq ? nxt : cur, pt, phys);
-                __syncwarp();
-                ++pt;
-                ++gi;
-                return true;
-            }
-            if (pq == 1 || exhausted) return false;
-            next_seg_item(a, starts, T, chunk, nw, stride, lane, s_hint, ps, nxt);
-            if (nxt.nt == 0) {
-                exhausted = true;
-                return false;
-            }
-            have_nxt = true;
-            pq = 1;
-            pt = 0;
-        }
-    };
-
-    if (!exhausted) {
-        while (gi - gc < (uint32_t)kStages && produce()) {
-        }
-    }
+    uint32_t gc = 0;
     const uint32_t slots_u32 = smem_u32(slots);
-    // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
-    // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
-    uint32_t qa0[8], qa2[8];
-    float m = -INFINITY, l = 0.f;  // row gq: running max (log2 units) and this lane's part of the sum
-    // O^T accumulators: o[mb] holds dims 16mb + gq (0, 1) and 16mb + gq + 8
-    // (2, 3) of query heads 2tq (0, 2) and 2tq + 1 (1, 3)
-    float o[8][4];
-    bool saw_bad = false;
-    while (cur.nt > 0) {
-        if (cur.first) {
+    // ldmatrix row addresses of this lane inside a K or V tile: row `key` of
+    // 16-byte chunk 2j + (q & 1) (j = ks & 3, plus 2048 for ks >= 4: the
+    // second 64-column box), 128-byte swizzle
+    uint32_t frag_off[4];
+    {
+        const int q = lane >> 3, key = 8 * (q >> 1) + (lane & 7);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) frag_off[j] = sw_off(key, 2 * j + (q & 1));
+    }
+    for (;;) {
+        SegItem cur;
+        next_seg_item(a, starts, T, chunk, nw, stride, s_hint, ps, cur);
+        if (cur.nt == 0) break;
+        // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
+        // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
+        uint32_t qa0[8], qa2[8];
+        {
             const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
                 a.q + ((size_t)cur.s * a.H + cur.h * G + (gq < G ? gq : 0)) * kD);
 #pragma unroll
@@ -933,20 +897,22 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                 qa0[ks] = gq < G ? __ldg(qrow + 8 * ks + tq) : 0u;
                 qa2[ks] = gq < G ? __ldg(qrow + 8 * ks + 4 + tq) : 0u;
             }
-            m = -INFINITY;
-            l = 0.f;
-#pragma unroll
-            for (int mb = 0; mb < 8; ++mb) o[mb][0] = o[mb][1] = o[mb][2] = o[mb][3] = 0.f;
-            saw_bad = false;
         }
-        for (int t = 0; t < cur.nt; ++t) {
+        float m = -INFINITY, l = 0.f;  // row gq: running max (log2 units) and this lane's part of the sum
+        // O^T accumulators: o[mb] holds dims 16mb + gq (0, 1) and 16mb + gq + 8
+        // (2, 3) of query heads 2tq (0, 2) and 2tq + 1 (1, 3)
+        float o[8][4];
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) o[mb][0] = o[mb][1] = o[mb][2] = o[mb][3] = 0.f;
+        bool saw_bad = false, dead = false;
+        for (int t = 0; t < cur.nt; ++t, ++gc) {
             const int slot = gc % kStages;
-            if (!mbar_wait(full + slot, (gc / kStages) & 1u, a.err)) {
+            if (!mbar_wait(my_full + slot, (gc / kStages) & 1u, a.err)) {
                 dead = true;
                 break;
             }
             const int tok = cur.tok0 + t * kTileTok;
-            const bool tile_ok = seg_tile_block(a, cur, t) >= 0;
+            const bool tile_ok = slot_bad[wid * kStages + slot] == 0;
             saw_bad |= !tile_ok;
             if (tile_ok) {
                 const uint32_t kt = slots_u32 + slot * kSlotBytes, vt = kt + kTileBytes;
@@ -959,19 +925,35 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                         const int r = valid + (e >> 4), c = e & 15;
                         *reinterpret_cast<uint4 *>(vrows + sw_off(r, c)) = make_uint4(0u, 0u, 0u, 0u);
                     }
+                    fence_proxy_async_smem();  // before the slot's next TMA refill
                     __syncwarp();
                 }
-                // S = Q K^T: keys 0..7 (n-block 0) and 8..15 (n-block 1)
+                // S = Q K^T: keys 0..7 (n-block 0) and 8..15 (n-block 1), the
+                // 128 dims in two independent halves (two shorter MMA chains);
+                // the asm statements keep their order, so every fragment load of
+                // the tile goes out before the first MMA that needs one
                 float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t vf[8][4];
                 {
-                    const int q = lane >> 3, i = lane & 7;
-                    const int key = 8 * (q >> 1) + i;
+                    uint32_t kf[8][4];
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        uint32_t b00, b01, b10, b11;
-                        ldsm_x4(kt + sw_off(key, 2 * ks + (q & 1)), b00, b01, b10, b11);
-                        mma_bf16(s0, qa0[ks], qa2[ks], b00, b01);
-                        mma_bf16(s1, qa0[ks], qa2[ks], b10, b11);
+                    for (int ks = 0; ks < 8; ++ks)
+                        ldsm_x4(kt + (ks >> 2) * 2048 + frag_off[ks & 3], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3]);
+#pragma unroll
+                    for (int mb = 0; mb < 8; ++mb)
+                        ldsm_x4_t(vt + (mb >> 2) * 2048 + frag_off[mb & 3], vf[mb][0], vf[mb][1], vf[mb][2], vf[mb][3]);
+                    float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        mma_bf16(s0, qa0[ks], qa2[ks], kf[ks][0], kf[ks][1]);
+                        mma_bf16(s1, qa0[ks], qa2[ks], kf[ks][2], kf[ks][3]);
+                        mma_bf16(u0, qa0[ks + 4], qa2[ks + 4], kf[ks + 4][0], kf[ks + 4][1]);
+                        mma_bf16(u1, qa0[ks + 4], qa2[ks + 4], kf[ks + 4][2], kf[ks + 4][3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        s0[e] += u0[e];
+                        s1[e] += u1[e];
                     }
                 }
                 // online softmax of row gq over the tile's 16 keys (this lane:
@@ -985,70 +967,129 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 1)
                 float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float m_new = fmaxf(m, mx);  // finite: key 0 of every tile is live
-                const float alpha = ex2_approx(m - m_new);
+                // lazy rescaling: the reference max moves only when the tile's
+                // max exceeds it by more than kLazyLog2 (always on the first
+                // tile, m = -inf); otherwise the probabilities are taken
+                // against the old max (at most 2^kLazyLog2) and nothing is
+                // rescaled -- O, l and the max stay consistent either way
+                const bool bump = mx > m + kLazyLog2;
+                const float m_new = bump ? mx : m;  // finite: key 0 of every tile is live
+                const float alpha = bump ? ex2_approx(m - m_new) : 1.f;
                 float p[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) p[e] = ex2_approx(x[e] - m_new);
                 l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
                 m = m_new;
-                // this lane's accumulators belong to query heads 2tq and 2tq + 1
-                const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * tq);
-                const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * tq + 4);
+                if (__any_sync(0xffffffffu, bump)) {
+                    // this lane's accumulators belong to query heads 2tq and 2tq + 1
+                    const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * tq);
+                    const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * tq + 4);
 #pragma unroll
-                for (int mb = 0; mb < 8; ++mb) {
-                    o[mb][0] *= al0;
-                    o[mb][2] *= al0;
-                    o[mb][1] *= al1;
-                    o[mb][3] *= al1;
+                    for (int mb = 0; mb < 8; ++mb) {
+                        o[mb][0] *= al0;
+                        o[mb][2] *= al0;
+                        o[mb][1] *= al1;
+                        o[mb][3] *= al1;
+                    }
                 }
                 // P^T fragments (keys 2tq, 2tq + 1 and 8 + 2tq, 9 + 2tq of head gq)
                 const uint32_t pb0 = pack_bf16x2(p[0], p[1]), pb1 = pack_bf16x2(p[2], p[3]);
                 // O^T += V^T P^T: dims 16mb .. 16mb + 15 per m-block
-                {
-                    const int q = lane >> 3, i = lane & 7;
-                    const int key = 8 * (q >> 1) + i;
 #pragma unroll
-                    for (int mb = 0; mb < 8; ++mb) {
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4_t(vt + sw_off(key, 2 * mb + (q & 1)), a0, a1, a2, a3);
-                        mma_bf16_4(o[mb], a0, a1, a2, a3, pb0, pb1);
-                    }
-                }
+                for (int mb = 0; mb < 8; ++mb) mma_bf16_4(o[mb], vf[mb][0], vf[mb][1], vf[mb][2], vf[mb][3], pb0, pb1);
             }
-            ++gc;
-            __syncwarp();  // every lane is done with the slot before it is refilled
-            if (gi - gc < (uint32_t)kStages) produce();
+            // the P V MMAs have issued, so every fragment load of the slot has
+            // completed: release it to the producer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(my_empty + slot);
         }
         if (dead) break;
-        if (cur.last) {
-            // unnormalised O rows -> per-warp scratch, then the common finish
-            // (final row, or partial + merge by the last segment)
-            float lt = l + __shfl_xor_sync(0xffffffffu, l, 1);
-            lt += __shfl_xor_sync(0xffffffffu, lt, 2);
-            if (2 * tq < G) {
+        // unnormalised O rows -> per-warp scratch, then the common finish
+        // (final row, or partial + merge by the last segment)
+        float lt = l + __shfl_xor_sync(0xffffffffu, l, 1);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+        if (2 * tq < G) {
 #pragma unroll
-                for (int mb = 0; mb < 8; ++mb) {
-                    scratch[(2 * tq) * kD + 16 * mb + gq] = o[mb][0];
-                    scratch[(2 * tq + 1) * kD + 16 * mb + gq] = o[mb][1];
-                    scratch[(2 * tq) * kD + 16 * mb + gq + 8] = o[mb][2];
-                    scratch[(2 * tq + 1) * kD + 16 * mb + gq + 8] = o[mb][3];
+            for (int mb = 0; mb < 8; ++mb) {
+                scratch[(2 * tq) * kD + 16 * mb + gq] = o[mb][0];
+                scratch[(2 * tq + 1) * kD + 16 * mb + gq] = o[mb][1];
+                scratch[(2 * tq) * kD + 16 * mb + gq + 8] = o[mb][2];
+                scratch[(2 * tq + 1) * kD + 16 * mb + gq + 8] = o[mb][3];
+            }
+        }
+        __syncwarp();
+        finish_seg<G>(a, cur, starts, chunk, lane, scratch, m, lt, saw_bad);
+        __syncwarp();  // scratch reads done before the next segment writes it
+    }
+}
+
+// The rows the grouped kernel left in partials, one warp per query head:
+// sh = s H + hq, key/value row r = s Hkv + hq / G, the row's segments in
+// slots slot0 .. slot0 + nsplit - 1 (slot0 = first worker + r).  Launched as
+// a programmatic dependent of decode_mma_kernel: griddepcontrol.wait returns
+// once that grid has finished and its writes are visible.  Lane j holds the
+// log2-sum-exps of partials j, j + 32, ...; the maximum and the weight sum
+// are warp reductions and the weighted rows are summed in partial order, so
+// the result depends only on the lengths and sizes.
+__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const long long sh = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (sh >= (long long)a.num_seqs * a.H) return;
+    const int s = (int)(sh / a.H), hq = (int)(sh - (long long)s * a.H);
+    const int h = hq / G, g = hq - h * G;
+    const int32_t *starts = a.item_start;
+    const int nts = starts[s + 1] - starts[s];
+    if (nts == 0) return;  // empty or invalid length: written by the plan
+    const long long T = (long long)starts[a.num_seqs] * a.Hkv;
+    const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
+    const long long row_begin = (long long)a.Hkv * starts[s] + (long long)h * nts;
+    const int w0 = (int)(row_begin / chunk);
+    const int nsplit = (int)((row_begin + nts - 1) / chunk) - w0 + 1;
+    if (nsplit == 1) return;  // written by its segment
+    if (__ldcg(a.seq_bad + s)) {
+        *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = make_uint2(0u, 0u);
+        if (lane == 0) a.LSE[sh] = -INFINITY;
+        return;
+    }
+    const size_t slot0 = (size_t)w0 + (size_t)s * a.Hkv + h;
+    const float *plse = a.part_lse + slot0 * G + g;                              // partial q at plse[q G]
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (slot0 * G + g) * kD) + lane;  // po[q G d / 4]
+    float M = -INFINITY;
+    for (int q = lane; q < nsplit; q += 32) M = fmaxf(M, __ldcg(plse + (size_t)q * G));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float tot = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q0 = 0; q0 < nsplit; q0 += 32) {
+        const int n = min(32, nsplit - q0);
+        const float wl = lane < n ? ex2_approx(__ldcg(plse + (size_t)(q0 + lane) * G) - M) : 0.f;
+        float part = wl;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        tot += part;
+        // the weighted rows in partial order, 8 loads in flight
+        for (int j0 = 0; j0 < n; j0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j0 + u < n) v[u] = __ldcg(po + (size_t)(q0 + j0 + u) * G * (kD / 4));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float w = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+                if (j0 + u < n) {
+                    acc.x = fmaf(w, v[u].x, acc.x);
+                    acc.y = fmaf(w, v[u].y, acc.y);
+                    acc.z = fmaf(w, v[u].z, acc.z);
+                    acc.w = fmaf(w, v[u].w, acc.w);
                 }
             }
-            __syncwarp();
-            finish_seg<G>(a, cur, lane, scratch, m, lt, saw_bad);
-            __syncwarp();  // scratch reads done before the next segment writes it
-        }
-        if (!have_nxt) break;
-        cur = nxt;
-        have_nxt = false;
-        pq = 0;
-        while (gi - gc < (uint32_t)kStages && produce()) {
         }
     }
-    if (dead && lane == 0) {
-        for (uint32_t g = gc; g < gi; ++g) mbar_wait(full + g % kStages, (g / kStages) & 1u, nullptr);
-    }
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (lane == 0) a.LSE[sh] = tot > 0.f ? (M + __log2f(tot)) * kLn2 : -INFINITY;
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -1072,11 +1113,11 @@ WsLayout ws_layout(int num_seqs, int H, size_t prow) {
 
 // Partial rows for these sizes: [num_seqs, H, max_splits] for the split
 // kernel; groups of 4 or more may run the scheduled kernel, whose slots hold
-// at most (kWorkers + num_seqs * H / G) x G rows (G <= 8 per slot).
+// at most (workers + num_seqs * H / G) x G rows (G <= 8 per slot).
 size_t partial_rows(int num_seqs, int H, int Hkv, int max_splits) {
     const size_t split_rows = (size_t)num_seqs * H * (size_t)(max_splits < 1 ? 1 : max_splits);
     if (H / Hkv < 4) return split_rows;
-    const size_t sched_rows = (size_t)kWorkers * 8 + (size_t)num_seqs * H;
+    const size_t sched_rows = (size_t)kMaxWorkers * 8 + (size_t)num_seqs * H;
     return split_rows > sched_rows ? split_rows : sched_rows;
 }
 
@@ -1149,7 +1190,7 @@ attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int 
         return ATTN_ECUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(kMmaWarps * 32);
+    cfg.blockDim = dim3(kMmaThreads);
     cfg.dynamicSmemBytes = kMmaSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1157,7 +1198,14 @@ attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<G>, tk, tv, a) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_mma_kernel<G>, tk, tv, a) != cudaSuccess) return ATTN_ECUDA;
+    // the rows left in partials, merged by a programmatic dependent
+    const long long rows_q = (long long)a.num_seqs * a.H;
+    cudaLaunchConfig_t mcfg = cfg;
+    mcfg.gridDim = dim3((unsigned)((rows_q + 7) / 8));
+    mcfg.blockDim = dim3(256);
+    mcfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&mcfg, decode_merge_kernel, a, G) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
@@ -1186,6 +1234,7 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.num_blocks = p.num_blocks;
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
+    a.bs_shift = p.block_size == 32 ? 5 : 4;
     if (G % 8 == 0 && G > 8) {
         // larger groups (multi-query attention): each cache head serves G / 8
         // virtual key/value heads of 8 query heads, adjacent in the schedule,

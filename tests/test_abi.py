@@ -124,7 +124,8 @@ def test_binding_refuses_cpu_tensors():
 def test_gqa_workspace_size(lib):
     """Grouped workspace: groups of 1 and 2 need the multi-head size; groups
     of 4 and more at least that and room for the balanced schedule's partial
-    rows (1480 runs x up to 8 heads + one per query head, d + 1 floats each),
+    rows (a bound of 1480 runs x up to 8 heads + one per query head, d + 1
+    floats each),
     which dominates for few short sequences; invalid groupings give 0."""
     mha = osp.paged_attn_decode_workspace_size(64, 32, 128, 256, 16)
     for hkv in (32, 16):

@@ -294,8 +294,8 @@ def test_gqa_long_row_many_segments(Hq, bs):
     """Groups of 4 and 8 run on a balanced schedule that cuts the (sequence,
     key/value head) rows into equal runs of tiles.  Few tiles in all give the
     shortest run (128 keys), so a 20000-token row is cut into more than 128
-    segments (the merge's many-partials path) beside short rows; a placement
-    shuffle is bit-identical."""
+    segments (the merge kernel's batches of 32 partials) beside short rows;
+    a placement shuffle is bit-identical."""
     lens = [20000, 1, 16, 17, 700]
     p = W.paged_uniform(H=1, d=128, block_size=bs, pool=1400, len_hi=20000, seed=90 + Hq, device="cuda", lens=lens)
     g = torch.Generator(device="cuda").manual_seed(91 + Hq)
@@ -312,7 +312,7 @@ def test_gqa_long_row_many_segments(Hq, bs):
 
 def test_gqa_odd_runs_cut_blocks():
     """64 sequences of 0..850 tokens, 8 key/value heads, G = 4, 32-token
-    blocks: 12776 tiles give runs of 9 tiles, so runs start and end in
+    blocks: 12776 tiles over 1184 workers give runs of 11 tiles, so runs start and end in
     the middle of cache blocks and rows; against the oracle, and a placement
     shuffle is bit-identical."""
     lens = np.random.default_rng(95).integers(0, 851, 64).tolist()  # lengths fixed on the host
@@ -320,7 +320,7 @@ def test_gqa_odd_runs_cut_blocks():
     g = torch.Generator(device="cuda").manual_seed(94)
     q = torch.randn((64, 32, 128), generator=g, device="cuda").to(torch.bfloat16)
     tiles = int(sum(-(-int(L) // 16) for L in lens)) * 8
-    assert -(-tiles // 1480) % 2 == 1, tiles  # an odd run length
+    assert -(-tiles // 1184) % 2 == 1, tiles  # an odd run length
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     O, LSE = _gqa(q, p, err)
     assert int(err.item()) == 0
