@@ -76,6 +76,7 @@ struct DecodeArgs {
     int32_t *item_start;  // [num_seqs + 1] prefix sum of splits per sequence
     int32_t *done_cnt;    // [num_seqs, H] splits finished per (sequence, head)
     int32_t *seq_bad;     // [num_seqs] nonzero: a block-table entry was out of range
+    int32_t *slot_bad;    // [partial slots] grouped kernel: the slot's segment met a bad block id
     float *part_lse;      // [num_seqs, H, max_splits] log2 units
     float *part_o;        // [num_seqs, H, max_splits, d] normalised
     int num_seqs, H, num_blocks, max_blocks, block_size, split_tokens, max_splits;
@@ -84,6 +85,7 @@ struct DecodeArgs {
     int kv_div;           // groups above 8 run as kv_div groups of 8 per cache head
     int bs_shift;         // log2(block_size)
     float scale_log2;     // scale * log2(e)
+    int fused_plan;       // grouped kernel: every CTA computes the plan itself (no plan kernel)
 };
 
 __device__ __forceinline__ bool seq_len_ok(int L, const DecodeArgs &a) {
@@ -756,7 +758,7 @@ __device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &i
             make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
     }
     if (lane < G) a.part_lse[(size_t)slot * G + lane] = lg_l > 0.f ? mg_l + __log2f(lg_l) : -INFINITY;
-    if (lane == 0 && saw_bad) atomicOr(a.seq_bad + s, 1);
+    if (lane == 0) a.slot_bad[slot] = saw_bad ? 1 : 0;  // written for every cut segment: nothing to clear
 }
 
 template <int G>
@@ -782,7 +784,51 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     pdl_wait();
     pdl_launch_dependents();  // the merge grid may be set up now; it waits for this grid's end
     const int32_t *starts = a.item_start;  // tiles before each sequence
-    if (a.num_seqs <= kMaxSmemSeqs) {
+    if (a.fused_plan) {
+        // the plan, in every CTA: tiles per sequence (none for an empty or
+        // invalid length) and their exclusive prefix, by a block-wide scan;
+        // CTA 0 publishes it for the merge kernel
+        __shared__ int warp_sum[kMmaThreads / 32];
+        int32_t *st = reinterpret_cast<int32_t *>(smem + kStartsOff);
+        const int n = a.num_seqs, per = (n + kMmaThreads - 1) / kMmaThreads;
+        const int k0 = min(n, (int)threadIdx.x * per), k1 = min(n, k0 + per);
+        auto seq_tiles = [&](int k) {
+            const int L = a.seq_lens[k];
+            return (L > 0 && seq_len_ok(L, a)) ? (L + kTileTok - 1) / kTileTok : 0;
+        };
+        int sum = 0;
+        for (int k = k0; k < k1; ++k) sum += seq_tiles(k);
+        int x = sum;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sum[wid] = x;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < wid; ++w) base += warp_sum[w];
+        int run = base + x - sum;
+        for (int k = k0; k < k1; ++k) {
+            st[k] = run;
+            run += seq_tiles(k);
+        }
+        if (threadIdx.x == kMmaThreads - 1) st[n] = base + x;
+        __syncthreads();
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i <= n; i += kMmaThreads) a.item_start[i] = st[i];
+        // empty and invalid sequences: O = 0, LSE = -inf (an invalid length
+        // also sets its error bit); sequences spread over the CTAs
+        for (int sq = blockIdx.x; sq < n; sq += gridDim.x) {
+            const int L = a.seq_lens[sq];
+            if (L > 0 && seq_len_ok(L, a)) continue;
+            if (threadIdx.x == 0 && !seq_len_ok(L, a) && a.err) atomicOr(a.err, ATTN_DEVERR_SEQ_LEN);
+            for (int e = threadIdx.x; e < a.H * (kD / 8); e += kMmaThreads)
+                reinterpret_cast<uint4 *>(a.O + (size_t)sq * a.H * kD)[e] = make_uint4(0u, 0u, 0u, 0u);
+            for (int hh = threadIdx.x; hh < a.H; hh += kMmaThreads) a.LSE[(size_t)sq * a.H + hh] = -INFINITY;
+        }
+        starts = st;
+    } else if (a.num_seqs <= kMaxSmemSeqs) {
         int32_t *st = reinterpret_cast<int32_t *>(smem + kStartsOff);
         for (int i = threadIdx.x; i <= a.num_seqs; i += blockDim.x) st[i] = a.item_start[i];
         starts = st;
@@ -1028,10 +1074,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 // slots slot0 .. slot0 + nsplit - 1 (slot0 = first worker + r).  Launched as
 // a programmatic dependent of decode_mma_kernel: griddepcontrol.wait returns
 // once that grid has finished and its writes are visible.  Lane j holds the
-// log2-sum-exps of partials j, j + 32, ...; the maximum and the weight sum
-// are warp reductions and the weighted rows are summed in partial order, so
-// the result depends only on the lengths and sizes.
+// log2-sum-exp and bad flag of partials j, j + 32, ...; the maximum and the
+// weight sum are warp reductions and the weighted rows are summed in partial
+// order, so the result depends only on the lengths and sizes.  The first 16
+// partial rows are requested together with the log2-sum-exps.
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) {
+    constexpr int kBatch = 16;  // partial rows in flight per lane
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long sh = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -1039,43 +1087,55 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) 
     const int s = (int)(sh / a.H), hq = (int)(sh - (long long)s * a.H);
     const int h = hq / G, g = hq - h * G;
     const int32_t *starts = a.item_start;
-    const int nts = starts[s + 1] - starts[s];
-    if (nts == 0) return;  // empty or invalid length: written by the plan
-    const long long T = (long long)starts[a.num_seqs] * a.Hkv;
+    const int st0 = __ldcg(starts + s), st1 = __ldcg(starts + s + 1), stn = __ldcg(starts + a.num_seqs);
+    const int nts = st1 - st0;
+    if (nts == 0) return;  // empty or invalid length: written with the plan
+    const long long T = (long long)stn * a.Hkv;
     const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
-    const long long row_begin = (long long)a.Hkv * starts[s] + (long long)h * nts;
+    const long long row_begin = (long long)a.Hkv * st0 + (long long)h * nts;
     const int w0 = (int)(row_begin / chunk);
     const int nsplit = (int)((row_begin + nts - 1) / chunk) - w0 + 1;
     if (nsplit == 1) return;  // written by its segment
-    if (__ldcg(a.seq_bad + s)) {
+    const size_t slot0 = (size_t)w0 + (size_t)s * a.Hkv + h;
+    const float *plse = a.part_lse + slot0 * G + g;                                      // partial q at plse[q G]
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (slot0 * G + g) * kD) + lane;  // po[q G d / 4]
+    const int32_t *pbad = a.slot_bad + slot0;
+    const float lse0 = lane < nsplit ? __ldcg(plse + (size_t)lane * G) : -INFINITY;
+    int bad = lane < nsplit ? __ldcg(pbad + lane) : 0;
+    float4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+        if (u < nsplit) v[u] = __ldcg(po + (size_t)u * G * (kD / 4));
+    float M = lse0;
+    for (int q = 32 + lane; q < nsplit; q += 32) {
+        M = fmaxf(M, __ldcg(plse + (size_t)q * G));
+        bad |= __ldcg(pbad + q);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (__any_sync(0xffffffffu, bad != 0)) {  // a bad block id in the row: the sequence's result is zeros
         *reinterpret_cast<uint2 *>(a.O + sh * kD + 4 * lane) = make_uint2(0u, 0u);
         if (lane == 0) a.LSE[sh] = -INFINITY;
         return;
     }
-    const size_t slot0 = (size_t)w0 + (size_t)s * a.Hkv + h;
-    const float *plse = a.part_lse + slot0 * G + g;                              // partial q at plse[q G]
-    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (slot0 * G + g) * kD) + lane;  // po[q G d / 4]
-    float M = -INFINITY;
-    for (int q = lane; q < nsplit; q += 32) M = fmaxf(M, __ldcg(plse + (size_t)q * G));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float tot = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int q0 = 0; q0 < nsplit; q0 += 32) {
         const int n = min(32, nsplit - q0);
-        const float wl = lane < n ? ex2_approx(__ldcg(plse + (size_t)(q0 + lane) * G) - M) : 0.f;
+        const float lse = q0 == 0 ? lse0 : (lane < n ? __ldcg(plse + (size_t)(q0 + lane) * G) : -INFINITY);
+        const float wl = lane < n ? ex2_approx(lse - M) : 0.f;
         float part = wl;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         tot += part;
-        // the weighted rows in partial order, 8 loads in flight
-        for (int j0 = 0; j0 < n; j0 += 8) {
-            float4 v[8];
+        for (int j0 = 0; j0 < n; j0 += kBatch) {
+            if (q0 + j0 > 0) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (j0 + u < n) v[u] = __ldcg(po + (size_t)(q0 + j0 + u) * G * (kD / 4));
+                for (int u = 0; u < kBatch; ++u)
+                    if (j0 + u < n) v[u] = __ldcg(po + (size_t)(q0 + j0 + u) * G * (kD / 4));
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < kBatch; ++u) {
                 const float w = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
                 if (j0 + u < n) {
                     acc.x = fmaf(w, v[u].x, acc.x);
@@ -1095,7 +1155,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t counter, item_start, done_cnt, seq_bad, part_lse, part_o, total;
+    size_t counter, item_start, done_cnt, seq_bad, slot_bad, part_lse, part_o, total;
 };
 
 // prow: partial rows (fp32 [d] each, plus a log2-sum-exp)
@@ -1105,7 +1165,8 @@ WsLayout ws_layout(int num_seqs, int H, size_t prow) {
     w.item_start = 256;
     w.done_cnt = align_up(w.item_start + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
     w.seq_bad = align_up(w.done_cnt + sizeof(int32_t) * (size_t)num_seqs * H, 256);
-    w.part_lse = align_up(w.seq_bad + sizeof(int32_t) * (size_t)num_seqs, 256);
+    w.slot_bad = align_up(w.seq_bad + sizeof(int32_t) * (size_t)num_seqs, 256);
+    w.part_lse = align_up(w.slot_bad + sizeof(int32_t) * (prow / 4 + 1), 256);  // slots hold >= 4 rows
     w.part_o = align_up(w.part_lse + sizeof(float) * prow, 256);
     w.total = align_up(w.part_o + sizeof(float) * prow * kD, 256);
     return w;
@@ -1259,11 +1320,16 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
     a.item_start = reinterpret_cast<int32_t *>(ws + w.item_start);
     a.done_cnt = reinterpret_cast<int32_t *>(ws + w.done_cnt);
     a.seq_bad = reinterpret_cast<int32_t *>(ws + w.seq_bad);
+    a.slot_bad = reinterpret_cast<int32_t *>(ws + w.slot_bad);
     a.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
     a.part_o = reinterpret_cast<float *>(ws + w.part_o);
 
-    decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    // the grouped kernel plans in every CTA when the offsets fit in shared memory
+    a.fused_plan = sched && p.num_seqs <= kMaxSmemSeqs ? 1 : 0;
+    if (!a.fused_plan) {
+        decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+    }
     if (sched) return G == 4 ? launch_mma<4>(a, p, dev, sm_count[dev], stream)
                              : launch_mma<8>(a, p, dev, sm_count[dev], stream);
     switch (G) {

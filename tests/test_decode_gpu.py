@@ -352,3 +352,28 @@ def test_gqa_bad_block_table_entry_in_cut_row(G):
     good = [0, 2, 3]
     O_ref, L_ref = _gqa_oracle(q, p, seqs=good)
     check_close(O[good], LSE[good], O_ref[good], L_ref[good], torch.bfloat16, f"G={G} good rows beside a bad one")
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_gqa_bad_seq_len_flags_and_zeroes(G):
+    """Grouped decode plans inside its own kernel: an invalid length (too long,
+    negative) still sets the error bit and zeroes that sequence, an empty one
+    is O = 0 / LSE = -inf without the bit, the others match the oracle."""
+    osp = _osp()
+    Hkv = 32 // G
+    lens = [300, 700, 0, 1500, 64]
+    p = W.paged_uniform(H=Hkv, d=128, block_size=16, pool=300, len_hi=1500, seed=97 + G, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(98 + G)
+    q = torch.randn((len(lens), 32, 128), generator=g, device="cuda").to(torch.bfloat16)
+    sl = p.seq_lens.clone()
+    sl[1] = p.block_table.shape[1] * 16 + 1
+    sl[4] = -3
+    bad = W.PagedInputs(q, p.k_cache, p.v_cache, p.block_table, sl, p.block_size, p.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _gqa(q, bad, err)
+    assert osp.attn_read_error(err) & osp.ATTN_DEVERR_SEQ_LEN
+    for s in (1, 2, 4):
+        assert (O[s] == 0).all() and torch.isneginf(LSE[s]).all()
+    good = [0, 3]
+    O_ref, L_ref = _gqa_oracle(q, p, seqs=good)
+    check_close(O[good], LSE[good], O_ref[good], L_ref[good], torch.bfloat16, f"G={G} good rows beside bad lengths")
