@@ -313,11 +313,13 @@ class Decode:
         self.ws = torch.empty(n, dtype=torch.uint8, device=device)
         self.ws_bytes = n
         self.unit, self.scale_unit = "GB/s", 1e9
-        # timed with its plan kernel (the events wrap the whole call); groups of
+        # timed as a whole call (the events wrap every kernel of it); groups of
         # 4 and 8 run the tensor-core variant and a merge kernel after it
         G = self.p.q.shape[1] // self.p.k_cache.shape[1]
         self.kernel = "decode_mma_kernel" if G >= 4 else "decode_split_kernel"
-        self.launches_per_step = 3 if G >= 4 else 2
+        # (groups of 4 and more plan inside their kernel up to 4096 sequences:
+        # that kernel and the merge; otherwise the plan kernel and one more)
+        self.launches_per_step = 2 + (1 if G >= 4 and self.p.num_seqs > 4096 else 0)
 
     def step(self, i, osp):
         p = self.p
