@@ -176,14 +176,40 @@ KERNEL_SOURCES = {"prefill_bf16_kernel": ("prefill_sm100.cu", "ptx.cuh", "launch
                   "block_copy_kernel": ("kv_cache_ops.cu", "ptx.cuh", "launch.h")}
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments, trailing blanks or empty lines (string
+    and character literals kept as written)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_sources_hash(kernel: str) -> str:
-    """Hash of the source files a kernel is built from (profiler counters are
-    only reported while these are unchanged)."""
+    """Hash of the code (comments and blank lines left out) of the source
+    files a kernel is built from: profiler counters are only reported while
+    it is unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "online_softmax_paged_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -31,7 +31,12 @@
 //                      warp that completes the last split of a (sequence,
 //                      head) merges them in split order:
 //                      LSE = log sum_p exp(LSE_p), O = sum_p e^{LSE_p-LSE} O_p.
-// Every arithmetic order depends only on logical token positions (which warp
+//   Grouped query heads (G = 4, 8, and groups of 8 above) take a third
+//   route, described at decode_mma_kernel: warp tensor-core MMAs per 16-key
+//   tile, a balanced static schedule of equal tile runs planned inside the
+//   kernel, a producer warp refilling each math warp's ring, and
+//   decode_merge_kernel for the rows the runs cut.
+// Every arithmetic order depends only on the lengths and sizes (which warp
 // runs a split, or merges, changes nothing), so moving blocks to other
 // physical ids gives bit-identical results.
 #include <cuda_runtime.h>
