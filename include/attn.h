@@ -347,6 +347,19 @@ ATTN_API attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_
  */
 ATTN_API attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream);
 
+/*
+ * Self-test of the failure path shared by every pipeline wait: launches one
+ * 32-thread CTA that waits, through the same bounded wait the kernels use,
+ * on an mbarrier phase that nothing completes.  After the wait limit (1 s of
+ * wall clock) the wait ORs ATTN_DEVERR_TIMEOUT into *err_flag (device int32,
+ * required) and gives up; *result (device int32, may be NULL) is set to 0 for
+ * "gave up", 1 for "completed" (never, here).  The kernel then returns
+ * normally, so the context stays usable.  Asynchronous on `stream`; for
+ * tests of error reporting (read the flag with attn_read_error).
+ * Errors: ATTN_EINVAL for a NULL or misaligned err_flag or result.
+ */
+ATTN_API attn_status attn_selftest_wait_timeout(int32_t *err_flag, int32_t *result, attn_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 ATTN_API const char *attn_status_str(attn_status s);
 

@@ -18,7 +18,7 @@ __all__ = [
     "paged_attn_decode_split_tokens", "paged_attn_decode_noalloc", "attn_read_error", "attn_status_str", "lib_path", "load",
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
     "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
-    "attn_quantize_fp8", "attn_fwd_fp8", "paged_attn_decode_gqa_workspace_size",
+    "attn_quantize_fp8", "attn_fwd_fp8", "paged_attn_decode_gqa_workspace_size", "attn_selftest_wait_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +35,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_
                     "attn_quantize_fp8", "attn_fwd_fp8",
                     "paged_kv_append",
                     "paged_block_copy",
-                    "attn_read_error", "attn_status_str")
+                    "attn_read_error", "attn_status_str", "attn_selftest_wait_timeout")
 
 # size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
 ATTN_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -94,6 +94,8 @@ def load():
     lib.paged_block_copy.restype = c_int
     lib.attn_read_error.argtypes = [vp, i32p, vp]
     lib.attn_read_error.restype = c_int
+    lib.attn_selftest_wait_timeout.argtypes = [vp, vp, vp]
+    lib.attn_selftest_wait_timeout.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
     lib.attn_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -398,6 +400,17 @@ def paged_block_copy(k_cache, v_cache, src_blocks, dst_blocks, err_flag=None, st
                                  _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_block_copy")
+
+
+def attn_selftest_wait_timeout(err_flag, result=None, stream=None) -> None:
+    """Launch the bounded-wait self-test (attn.h): one CTA waits on an
+    mbarrier phase nothing completes; after the 1 s limit the wait ORs
+    ATTN_DEVERR_TIMEOUT into ``err_flag`` (int32 CUDA tensor) and writes 0 to
+    ``result`` (int32 CUDA tensor, optional).  Asynchronous."""
+    _check_cuda(err_flag, result)
+    st = load().attn_selftest_wait_timeout(_ptr(err_flag), _ptr(result), _stream(stream, err_flag.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_wait_timeout")
 
 
 def attn_read_error(err_flag, stream=None) -> int:

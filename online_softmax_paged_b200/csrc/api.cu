@@ -9,6 +9,11 @@
 #include "../../include/attn.h"
 #include "launch.h"
 
+namespace osp {
+// One CTA waits on an mbarrier phase that never completes (selftest.cu).
+attn_status launch_wait_timeout_selftest(int32_t *err_flag, int32_t *result, cudaStream_t stream);
+}  // namespace osp
+
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -190,6 +195,11 @@ attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_t *src_bl
     osp::CopyLaunch p{k_cache, v_cache, src_blocks, dst_blocks, num_pairs, num_blocks, H, d, block_size,
                       dt == ATTN_BF16 ? 2 : 4, err_flag};
     return osp::launch_block_copy(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_selftest_wait_timeout(int32_t *err_flag, int32_t *result, attn_stream_t stream) {
+    if (!err_flag || ((uintptr_t)err_flag & 3u) || ((uintptr_t)result & 3u)) return ATTN_EINVAL;
+    return osp::launch_wait_timeout_selftest(err_flag, result, reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream) {
