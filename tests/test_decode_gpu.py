@@ -182,7 +182,7 @@ def test_decode_equals_dense_last_row():
     assert (LSE[0] - Ld[0, :, L - 1]).abs().max().item() <= 1e-3
 
 
-@pytest.mark.parametrize("G,bs", [(2, 16), (4, 32), (8, 16), (4, 16)])
+@pytest.mark.parametrize("G,bs", [(2, 16), (4, 32), (8, 16), (4, 16), (8, 32), (2, 32)])
 def test_gqa_decode_full(G, bs):
     """Grouped-query decode: H_q = 32 query heads over 32 / G key/value heads,
     lengths 0..3000 (edge lengths included), against the grouped oracle."""
@@ -377,3 +377,23 @@ def test_gqa_bad_seq_len_flags_and_zeroes(G):
     good = [0, 3]
     O_ref, L_ref = _gqa_oracle(q, p, seqs=good)
     check_close(O[good], LSE[good], O_ref[good], L_ref[good], torch.bfloat16, f"G={G} good rows beside bad lengths")
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_gqa_many_sequences_plan_kernel(G):
+    """Above 4096 sequences the grouped kernel takes its offsets from the
+    plan kernel (global memory) instead of planning in shared memory: 4100
+    short sequences (0..40 tokens, some empty), against the oracle, and a
+    placement shuffle is bit-identical."""
+    lens = np.random.default_rng(120 + G).integers(0, 41, 4100).tolist()
+    p = W.paged_uniform(H=8 // G, d=128, block_size=16, pool=12400, len_hi=40, seed=121 + G, device="cuda", lens=lens)
+    g = torch.Generator(device="cuda").manual_seed(122 + G)
+    q = torch.randn((len(lens), 8, 128), generator=g, device="cuda").to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, LSE = _gqa(q, p, err)
+    assert int(err.item()) == 0
+    O_ref, L_ref = _gqa_oracle(q, p)
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"4100 sequences G={G}")
+    p2 = W.shuffle_placement(p, seed=9)
+    O2, L2 = _gqa(q, p2)
+    assert torch.equal(O, O2) and torch.equal(LSE, L2)
