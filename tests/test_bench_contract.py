@@ -28,3 +28,23 @@ def test_reference_arm_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
+
+
+def test_traffic_records_follow_code_not_comments():
+    """Recorded DRAM traffic is reported only while the kernel's code is the
+    one it was measured on: the source hash ignores comments and blank lines
+    but not code, string literals included."""
+    sys.path.insert(0, ROOT)
+    import bench
+    base = 'int a = 1; // note\n/* block\n comment */\nconst char *s = "x//y";\n\n'
+    assert bench._code_only(base) == bench._code_only(base.replace("// note", "// other note") + "\n\n// tail")
+    assert bench._code_only(base) != bench._code_only(base.replace("a = 1", "a = 2"))
+    assert bench._code_only(base) != bench._code_only(base.replace('"x//y"', '"x//z"'))
+    assert '"x//y"' in bench._code_only(base)
+    # every record names the kernel's current code (no stale record on file)
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        records = json.load(f)
+    for key, rec in records.items():
+        kernel, workload = key.split(":")
+        assert rec["sources"] == bench.kernel_sources_hash(kernel), key
+        assert bench.recorded_traffic(kernel, workload) == rec["bytes_per_launch"], key
