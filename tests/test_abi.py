@@ -137,3 +137,43 @@ def test_gqa_workspace_size(lib):
     assert small >= (1480 * 8 + 8) * 129 * 4
     assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 3, 128, 256, 16) == 0
     assert osp.paged_attn_decode_gqa_workspace_size(64, 32, 0, 128, 256, 16) == 0
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "attn.h"
+
+/* A plain C caller: no CUDA or PyTorch headers, only the library's. */
+int main(void) {
+    size_t ws = paged_attn_decode_workspace_size(64, 32, 128, 256, 16);
+    size_t wg = paged_attn_decode_gqa_workspace_size(64, 32, 4, 128, 256, 16);
+    int split = paged_attn_decode_split_tokens(64, 32, 128, 256, 16);
+    /* host-side argument checks reject these before any CUDA call */
+    attn_status s1 = attn_fwd(0, 0, 0, 0, 0, 1, 1, 1, 128, 0, 0.1f, ATTN_BF16, 0, 0);
+    attn_status s2 = paged_attn_decode(0, 0, 0, 0, 0, 16, 0, 0, 1, 1, 128, 1, 1, 0.1f, ATTN_BF16, 0, 0, 0, 0);
+    attn_status s3 = attn_selftest_wait_timeout(0, 0, 0);
+    printf("%zu %zu %d %s %s %s\n", ws, wg, split, attn_status_str(s1), attn_status_str(s2), attn_status_str(s3));
+    return (ws > 0 && wg >= ws && split > 0 && s1 == ATTN_EINVAL && s2 == ATTN_EINVAL && s3 == ATTN_EINVAL) ? 0 : 1;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    """The header is C99 (warnings as errors) and a C program links against
+    the library with nothing but it; the host-only calls run without a GPU."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(osp.lib_path())
+    libname = os.path.basename(osp.lib_path())
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                         str(src), "-o", str(exe), os.path.join(libdir, libname), "-Wl,-rpath," + libdir],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    fields = run.stdout.split()
+    assert int(fields[0]) == osp.paged_attn_decode_workspace_size(64, 32, 128, 256, 16)
+    # the library needs no PyTorch: its dynamic dependencies are system ones
+    deps = subprocess.run(["ldd", osp.lib_path()], capture_output=True, text=True).stdout
+    assert "torch" not in deps and "c10" not in deps, deps
