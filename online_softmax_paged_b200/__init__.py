@@ -19,6 +19,7 @@ __all__ = [
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
     "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
     "attn_quantize_fp8", "attn_fwd_fp8", "paged_attn_decode_gqa_workspace_size", "attn_selftest_wait_timeout",
+    "attn_selftest_exp2_poly",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +36,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_
                     "attn_quantize_fp8", "attn_fwd_fp8",
                     "paged_kv_append",
                     "paged_block_copy",
-                    "attn_read_error", "attn_status_str", "attn_selftest_wait_timeout")
+                    "attn_read_error", "attn_status_str", "attn_selftest_wait_timeout", "attn_selftest_exp2_poly")
 
 # size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
 ATTN_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -96,6 +97,8 @@ def load():
     lib.attn_read_error.restype = c_int
     lib.attn_selftest_wait_timeout.argtypes = [vp, vp, vp]
     lib.attn_selftest_wait_timeout.restype = c_int
+    lib.attn_selftest_exp2_poly.argtypes = [vp, vp, c_int, vp]
+    lib.attn_selftest_exp2_poly.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
     lib.attn_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -122,6 +125,30 @@ def _check_cuda(*ts):
             raise ValueError("all tensors must be on a CUDA device (the library has no CPU path)")
 
 
+def _check_device(dev, *ts):
+    """Every given tensor must be on ``dev``: the library launches on the
+    device that holds the inputs and reads every pointer there."""
+    for t in ts:
+        if t is not None and t.device != dev:
+            raise ValueError(f"all tensors must be on {dev} (got one on {t.device})")
+
+
+def _check_tensor(t, shape, dtype, name):
+    """``t`` (when given) must be a contiguous ``dtype`` tensor of ``shape``:
+    the kernels index it by the sizes passed, so anything smaller would be
+    read or written past its end."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} "
+                         f"(got {t.dtype} {tuple(t.shape)}{'' if t.is_contiguous() else ', not contiguous'})")
+
+
+def _check_err_flag(err_flag):
+    if err_flag is not None and (err_flag.dtype != torch.int32 or err_flag.numel() < 1):
+        raise ValueError("err_flag must be an int32 tensor with at least one element")
+
+
 def _dtype_code(dt):
     if dt == torch.bfloat16:
         return ATTN_BF16
@@ -140,14 +167,19 @@ def attn_fwd(Q, K, V, O=None, LSE=None, causal=False, scale=None, err_flag=None,
         raise ValueError("Q, K, V must share shape and dtype")
     if not (Q.is_contiguous() and K.is_contiguous() and V.is_contiguous()):
         raise ValueError("Q, K, V must be contiguous")
+    _check_device(Q.device, K, V, O, LSE, err_flag)
+    _check_tensor(O, Q.shape, Q.dtype, "O")
+    _check_tensor(LSE, (B, H, N), torch.float32, "LSE")
+    _check_err_flag(err_flag)
     if O is None:
         O = torch.empty_like(Q)
     if LSE is None:
         LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    st = load().attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, int(bool(causal)),
-                         float(scale), _dtype_code(Q.dtype), _ptr(err_flag), _stream(stream, Q.device))
+    with torch.cuda.device(Q.device):
+        st = load().attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, int(bool(causal)),
+                             float(scale), _dtype_code(Q.dtype), _ptr(err_flag), _stream(stream, Q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
     return O, LSE
@@ -165,13 +197,18 @@ def attn_quantize_fp8(x, signs=None, codes=None, scales=None, stream=None):
     *lead, N, d = x.shape
     BH = int(math.prod(lead)) if lead else 1
     nblk = -(-N // 128)
+    _check_device(x.device, signs, codes, scales)
+    _check_tensor(codes, x.shape, torch.uint8, "codes")
+    _check_tensor(scales, tuple(lead) + (nblk,), torch.float32, "scales")
     if codes is None:
         codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(tuple(lead) + (nblk,), dtype=torch.float32, device=x.device)
-    if signs is not None and (signs.dtype != torch.int8 or signs.numel() != d):
-        raise ValueError("signs must be d int8 values")
-    st = load().attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(scales), BH, N, d, _ptr(signs), _stream(stream, x.device))
+    if signs is not None and (signs.dtype != torch.int8 or signs.numel() != d or not signs.is_contiguous()):
+        raise ValueError("signs must be d contiguous int8 values")
+    with torch.cuda.device(x.device):
+        st = load().attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(scales), BH, N, d, _ptr(signs),
+                                      _stream(stream, x.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_quantize_fp8")
     return codes, scales
@@ -192,19 +229,59 @@ def attn_fwd_fp8(q8, q_scale, k8, k_scale, V, O=None, LSE=None, causal=False, sc
         if not t.is_contiguous():
             raise ValueError("inputs must be contiguous")
     nblk = -(-N // 128)
-    if q_scale.shape != (B, H, nblk) or k_scale.shape != (B, H, nblk):
-        raise ValueError("scales must be [B, H, ceil(N / 128)]")
+    _check_tensor(q_scale, (B, H, nblk), torch.float32, "q_scale")
+    _check_tensor(k_scale, (B, H, nblk), torch.float32, "k_scale")
+    _check_device(V.device, q8, q_scale, k8, k_scale, O, LSE, err_flag)
+    _check_tensor(O, V.shape, torch.bfloat16, "O")
+    _check_tensor(LSE, (B, H, N), torch.float32, "LSE")
+    _check_err_flag(err_flag)
     if O is None:
         O = torch.empty_like(V)
     if LSE is None:
         LSE = torch.empty((B, H, N), dtype=torch.float32, device=V.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    st = load().attn_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(V), _ptr(O), _ptr(LSE), B, H,
-                             N, d, int(bool(causal)), float(scale), _ptr(err_flag), _stream(stream, V.device))
+    with torch.cuda.device(V.device):
+        st = load().attn_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(V), _ptr(O), _ptr(LSE), B,
+                                 H, N, d, int(bool(causal)), float(scale), _ptr(err_flag), _stream(stream, V.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_fp8")
     return O, LSE
+
+
+def _check_decode_args(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE, err_flag, grouped):
+    """Shapes, dtypes, layout and device of a paged decode call's tensors.
+    Returns (S, H_q, H_kv, d, num_blocks, max_blocks_per_seq)."""
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [S, H, d] and the caches [num_blocks, H_kv, block_size, d]")
+    S, Hq, d = q.shape
+    nb, Hkv, bs, dk = k_cache.shape
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if k_cache.shape != v_cache.shape or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype or \
+            bs != block_size or dk != d or (not grouped and Hkv != Hq):
+        raise ValueError("caches must be [num_blocks, H, block_size, d] of q's dtype"
+                         + (" (H = H_kv)" if grouped else ""))
+    if block_table.dim() != 2 or block_table.shape[0] != S:
+        raise ValueError(f"block_table must be [S, max_blocks_per_seq] with S = {S}")
+    if tuple(seq_lens.shape) != (S,):
+        raise ValueError(f"seq_lens must hold S = {S} lengths")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    _check_device(q.device, k_cache, v_cache, block_table, seq_lens, O, LSE, err_flag)
+    _check_tensor(O, q.shape, q.dtype, "O")
+    _check_tensor(LSE, (S, Hq), torch.float32, "LSE")
+    _check_err_flag(err_flag)
+    return S, Hq, Hkv, d, nb, block_table.shape[1]
+
+
+def _check_workspace(workspace, dev):
+    if workspace is None:
+        return
+    _check_device(dev, workspace)
+    if not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
 
 
 def paged_attn_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq, block_size) -> int:
@@ -227,30 +304,24 @@ def paged_attn_decode(q, k_cache, v_cache, block_table, seq_lens, block_size, O=
     Returns (O, LSE).  ``workspace`` (uint8 CUDA tensor) is allocated when
     not given.  See ``paged_attn_decode`` in include/attn.h."""
     _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, workspace, err_flag)
-    S, H, d = q.shape
-    num_blocks = k_cache.shape[0]
-    mb = block_table.shape[1]
-    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
-        raise ValueError("block_table and seq_lens must be int32")
-    if k_cache.shape != v_cache.shape or k_cache.shape[1] != H or k_cache.shape[2] != block_size or \
-            k_cache.shape[3] != d:
-        raise ValueError("caches must be [num_blocks, H, block_size, d]")
-    for t in (q, k_cache, v_cache, block_table, seq_lens):
-        if not t.is_contiguous():
-            raise ValueError("inputs must be contiguous")
+    S, H, _, d, num_blocks, mb = _check_decode_args(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE,
+                                                    err_flag, grouped=False)
+    _check_workspace(workspace, q.device)
     if O is None:
         O = torch.empty_like(q)
     if LSE is None:
         LSE = torch.empty((S, H), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if workspace is None:  # (a given workspace is checked against the need by the library)
-        need = paged_attn_decode_workspace_size(S, H, d, mb, block_size)
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    st = load().paged_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
-                                  int(block_size), _ptr(O), _ptr(LSE), S, H, d, num_blocks, mb, float(scale),
-                                  _dtype_code(q.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                  _ptr(err_flag), _stream(stream, q.device))
+    with torch.cuda.device(q.device):
+        if workspace is None:  # (a given workspace is checked against the need by the library)
+            need = paged_attn_decode_workspace_size(S, H, d, mb, block_size)
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        st = load().paged_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                      int(block_size), _ptr(O), _ptr(LSE), S, H, d, num_blocks, mb, float(scale),
+                                      _dtype_code(q.dtype), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _ptr(err_flag),
+                                      _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode")
     return O, LSE
@@ -262,30 +333,24 @@ def paged_attn_decode_gqa(q, k_cache, v_cache, block_table, seq_lens, block_size
     block_size, d] with H_q / H_kv in {1, 2, 4} or a multiple of 8 (H_kv = 1:
     multi-query attention).  See include/attn.h."""
     _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, workspace, err_flag)
-    S, Hq, d = q.shape
-    nb, Hkv, bs, dk = k_cache.shape
-    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
-        raise ValueError("block_table and seq_lens must be int32")
-    if k_cache.shape != v_cache.shape or bs != block_size or dk != d:
-        raise ValueError("caches must be [num_blocks, H_kv, block_size, d]")
-    for t in (q, k_cache, v_cache, block_table, seq_lens):
-        if not t.is_contiguous():
-            raise ValueError("inputs must be contiguous")
+    S, Hq, Hkv, d, nb, mb = _check_decode_args(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE,
+                                               err_flag, grouped=True)
+    _check_workspace(workspace, q.device)
     if O is None:
         O = torch.empty_like(q)
     if LSE is None:
         LSE = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    mb = block_table.shape[1]
-    if workspace is None:  # (a given workspace is checked against the need by the library)
-        need = paged_attn_decode_gqa_workspace_size(S, Hq, Hkv, d, mb, block_size)
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    st = load().paged_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
-                                      int(block_size), _ptr(O), _ptr(LSE), S, Hq, Hkv, d, nb, mb, float(scale),
-                                      _dtype_code(q.dtype), _ptr(workspace),
-                                      workspace.numel() * workspace.element_size(), _ptr(err_flag),
-                                      _stream(stream, q.device))
+    with torch.cuda.device(q.device):
+        if workspace is None:  # (a given workspace is checked against the need by the library)
+            need = paged_attn_decode_gqa_workspace_size(S, Hq, Hkv, d, mb, block_size)
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        st = load().paged_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                          _ptr(seq_lens), int(block_size), _ptr(O), _ptr(LSE), S, Hq, Hkv, d, nb, mb,
+                                          float(scale), _dtype_code(q.dtype), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _ptr(err_flag),
+                                          _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode_gqa")
     return O, LSE
@@ -309,9 +374,17 @@ def paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_s
         raise ValueError("cu_q must be [S + 1] and block_table [S, max_blocks]")
     if k_cache.shape != v_cache.shape or bs != block_size or dk != d:
         raise ValueError("caches must be [num_blocks, H_kv, block_size, d]")
+    if block_table.dim() != 2 or tuple(seq_lens.shape) != (S,):
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("caches must have q's dtype")
     for t in (q, k_cache, v_cache, block_table, seq_lens, cu_q):
         if not t.is_contiguous():
             raise ValueError("inputs must be contiguous")
+    _check_device(q.device, k_cache, v_cache, block_table, seq_lens, cu_q, O, LSE, err_flag)
+    _check_tensor(O, q.shape, q.dtype, "O")
+    _check_tensor(LSE, (T, Hq), torch.float32, "LSE")
+    _check_err_flag(err_flag)
     if max_q_per_seq is None:
         max_q_per_seq = int((cu_q[1:] - cu_q[:-1]).max().item()) if S > 0 else 0
     if O is None:
@@ -320,10 +393,11 @@ def paged_attn_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_s
         LSE = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    st = load().paged_attn_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
-                                   _ptr(cu_q), int(block_size), _ptr(O), _ptr(LSE), S, T, int(max_q_per_seq), Hq,
-                                   Hkv, d, nb, block_table.shape[1], float(scale), _dtype_code(q.dtype),
-                                   _ptr(err_flag), _stream(stream, q.device))
+    with torch.cuda.device(q.device):
+        st = load().paged_attn_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                       _ptr(cu_q), int(block_size), _ptr(O), _ptr(LSE), S, T, int(max_q_per_seq),
+                                       Hq, Hkv, d, nb, block_table.shape[1], float(scale), _dtype_code(q.dtype),
+                                       _ptr(err_flag), _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_prefill")
     return O, LSE
@@ -340,25 +414,20 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, block_
     nothing).  Raises AttnError (ATTN_EUNSUPPORTED) when the sizes need more
     scratch than the array holds."""
     _check_cuda(q, k_cache, v_cache, block_table, seq_lens, O, LSE, err_flag)
-    S, H, d = q.shape
-    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
-        raise ValueError("block_table and seq_lens must be int32")
-    if k_cache.shape != v_cache.shape or k_cache.shape[1] != H or k_cache.shape[2] != block_size or \
-            k_cache.shape[3] != d:
-        raise ValueError("caches must be [num_blocks, H, block_size, d]")
-    for t in (q, k_cache, v_cache, block_table, seq_lens):
-        if not t.is_contiguous():
-            raise ValueError("inputs must be contiguous")
+    S, H, _, d, nb, mb = _check_decode_args(q, k_cache, v_cache, block_table, seq_lens, block_size, O, LSE,
+                                            err_flag, grouped=False)
     if O is None:
         O = torch.empty_like(q)
     if LSE is None:
         LSE = torch.empty((S, H), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    st = load().paged_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
-                                          _ptr(seq_lens), int(block_size), _ptr(O), _ptr(LSE), S, H, d,
-                                          k_cache.shape[0], block_table.shape[1], float(scale),
-                                          _dtype_code(q.dtype), _ptr(err_flag), _stream(stream, q.device))
+    # the library picks the scratch array of the current device: make it q's
+    with torch.cuda.device(q.device):
+        st = load().paged_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                              _ptr(seq_lens), int(block_size), _ptr(O), _ptr(LSE), S, H, d, nb, mb,
+                                              float(scale), _dtype_code(q.dtype), _ptr(err_flag),
+                                              _stream(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_attn_decode_noalloc (scratch limit %d bytes)" % ATTN_NOALLOC_SCRATCH_BYTES)
     return O, LSE
@@ -375,13 +444,18 @@ def paged_kv_append(k_new, v_new, seq_ids, positions, block_table, k_cache, v_ca
         raise ValueError("k_new/v_new [T, H, d] and caches [num_blocks, H, block_size, d] of one dtype")
     if seq_ids.dtype != torch.int32 or positions.dtype != torch.int32 or block_table.dtype != torch.int32:
         raise ValueError("seq_ids, positions and block_table must be int32")
+    if tuple(seq_ids.shape) != (T,) or tuple(positions.shape) != (T,) or block_table.dim() != 2:
+        raise ValueError("seq_ids and positions must be [T] and block_table [S, max_blocks_per_seq]")
     for t in (k_new, v_new, seq_ids, positions, block_table, k_cache, v_cache):
         if not t.is_contiguous():
             raise ValueError("inputs must be contiguous")
-    st = load().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(seq_ids), _ptr(positions), T, _ptr(block_table),
-                                block_table.shape[0], block_table.shape[1], _ptr(k_cache), _ptr(v_cache),
-                                k_cache.shape[0], H, d, k_cache.shape[2], _dtype_code(k_cache.dtype),
-                                _ptr(err_flag), _stream(stream, k_cache.device))
+    _check_device(k_cache.device, k_new, v_new, seq_ids, positions, block_table, v_cache, err_flag)
+    _check_err_flag(err_flag)
+    with torch.cuda.device(k_cache.device):
+        st = load().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(seq_ids), _ptr(positions), T,
+                                    _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(k_cache),
+                                    _ptr(v_cache), k_cache.shape[0], H, d, k_cache.shape[2],
+                                    _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_kv_append")
 
@@ -394,10 +468,15 @@ def paged_block_copy(k_cache, v_cache, src_blocks, dst_blocks, err_flag=None, st
         raise ValueError("src_blocks and dst_blocks: int32 of one length")
     if k_cache.shape != v_cache.shape or not (k_cache.is_contiguous() and v_cache.is_contiguous()):
         raise ValueError("caches must be contiguous [num_blocks, H, block_size, d] of one shape")
+    if v_cache.dtype != k_cache.dtype or k_cache.dim() != 4:
+        raise ValueError("caches must be [num_blocks, H, block_size, d] of one dtype")
+    _check_device(k_cache.device, v_cache, src_blocks, dst_blocks, err_flag)
+    _check_err_flag(err_flag)
     nb, H, bs, d = k_cache.shape
-    st = load().paged_block_copy(_ptr(k_cache), _ptr(v_cache), _ptr(src_blocks.contiguous()),
-                                 _ptr(dst_blocks.contiguous()), src_blocks.numel(), nb, H, d, bs,
-                                 _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
+    src, dst = src_blocks.contiguous(), dst_blocks.contiguous()
+    with torch.cuda.device(k_cache.device):
+        st = load().paged_block_copy(_ptr(k_cache), _ptr(v_cache), _ptr(src), _ptr(dst), src.numel(), nb, H, d,
+                                     bs, _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_block_copy")
 
@@ -408,15 +487,41 @@ def attn_selftest_wait_timeout(err_flag, result=None, stream=None) -> None:
     ATTN_DEVERR_TIMEOUT into ``err_flag`` (int32 CUDA tensor) and writes 0 to
     ``result`` (int32 CUDA tensor, optional).  Asynchronous."""
     _check_cuda(err_flag, result)
-    st = load().attn_selftest_wait_timeout(_ptr(err_flag), _ptr(result), _stream(stream, err_flag.device))
+    _check_err_flag(err_flag)
+    _check_device(err_flag.device, result)
+    if result is not None and (result.dtype != torch.int32 or result.numel() < 1):
+        raise ValueError("result must be an int32 tensor with at least one element")
+    with torch.cuda.device(err_flag.device):
+        st = load().attn_selftest_wait_timeout(_ptr(err_flag), _ptr(result), _stream(stream, err_flag.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_selftest_wait_timeout")
 
 
+def attn_selftest_exp2_poly(x, y=None, stream=None):
+    """The prefill kernel's FMA-pipe 2^x on the fp32 CUDA tensor ``x``
+    (attn.h: relative error <= 7.5e-5 on [-125, 8]).  Returns y (allocated
+    when not given).  Asynchronous."""
+    _check_cuda(x, y)
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 tensor")
+    _check_device(x.device, y)
+    _check_tensor(y, x.shape, torch.float32, "y")
+    if y is None:
+        y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        st = load().attn_selftest_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_exp2_poly")
+    return y
+
+
 def attn_read_error(err_flag, stream=None) -> int:
     """Synchronise the stream and return the device error bits (0 = none)."""
+    _check_cuda(err_flag)
+    _check_err_flag(err_flag)
     bits = ctypes.c_int32(0)
-    st = load().attn_read_error(_ptr(err_flag), ctypes.byref(bits), _stream(stream, err_flag.device))
+    with torch.cuda.device(err_flag.device):
+        st = load().attn_read_error(_ptr(err_flag), ctypes.byref(bits), _stream(stream, err_flag.device))
     if st not in (ATTN_OK, ATTN_EDEVICE):
         raise AttnError(st, "attn_read_error")
     return int(bits.value)

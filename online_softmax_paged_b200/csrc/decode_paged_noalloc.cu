@@ -18,9 +18,15 @@
 //   * All calls on a device share the one array.  Two calls whose kernels
 //     overlap on the GPU (different streams without ordering between them)
 //     race on it and give wrong results; calls on one stream are ordered.
-//   * The array keeps whatever the previous call left there.  The only part
-//     that must start at zero -- the work counter -- is zeroed by the first
-//     kernel of every call; every other byte is written before it is read.
+//   * The array keeps whatever the previous call left there.  Three areas of
+//     it must start at zero: the work counter, the per-(sequence, head)
+//     completion counts (done_cnt) and the per-sequence bad-block marks
+//     (seq_bad).  decode_plan_kernel, the first kernel of every call,
+//     clears all three; every other byte is written before it is read.  A
+//     change that adds another counter must clear it there too.
+//   * The scratch used is the current device's: the tensors' device must be
+//     current when the function is called (the address of another device's
+//     array would be read as garbage on this one).
 //   * The scratch address is looked up once per device, on the first call
 //     made while that device is current.  Make that first call before any
 //     stream capture begins, since the lookup is a runtime call.

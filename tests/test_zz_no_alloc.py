@@ -6,14 +6,18 @@ scratch array compiled into the library instead.
 
 Checked through the C ABI against the workspace-taking entry point on two
 calls in a row with different inputs (the second call runs on whatever the
-first left in the shared scratch), and that sizes too large for the scratch
-are refused.  This file is named to be collected last.
+first left in the shared scratch).  Both entry points run the same plan and
+kernels on the same sizes, so O and LSE must be bit-identical, not merely
+close; each call is also compared with the oracle on sampled sequences.
+Sizes too large for the scratch are refused.  This file is named to be
+collected last.
 """
 import pytest
 import torch
 
+import oracle
 import workloads as W
-from tests._parity import check_close, to64
+from tests._parity import DeviceCache, check_close, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -41,9 +45,15 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
                             device="cuda")
     second = W.paged_uniform(num_seqs=19, H=8, d=128, block_size=32, pool=3000, len_lo=0, len_hi=3000, seed=5,
                              device="cuda")
-    for name, p in (("first", first), ("second", second)):
-        O, L, O_ref, L_ref = _both(osp, p)
-        check_close(O, L, to64(O_ref), to64(L_ref), torch.bfloat16, f"no-alloc vs workspace ({name} call)")
+    for name, p, seqs in (("first", first, [0, 17, 40, 63]), ("second", second, list(range(19)))):
+        O, L, O_ws, L_ws = _both(osp, p)
+        # same plan, same kernels, same sizes: identical bits
+        assert torch.equal(O, O_ws), f"{name} call: O differs from the workspace entry point"
+        assert torch.equal(L, L_ws), f"{name} call: LSE differs from the workspace entry point"
+        O_ref, L_ref = oracle.paged_decode(to64(p.q), DeviceCache(p.k_cache), DeviceCache(p.v_cache),
+                                           p.block_table.cpu().numpy(), p.seq_lens.cpu().numpy(), p.block_size,
+                                           p.scale, seqs=seqs)
+        check_close(O[seqs], L[seqs], O_ref[seqs], L_ref[seqs], torch.bfloat16, f"no-alloc vs oracle ({name} call)")
 
 
 def test_noalloc_refuses_sizes_beyond_scratch():
