@@ -284,7 +284,10 @@ ATTN_API attn_status paged_attn_prefill(const void *q, const void *k_cache, cons
  *     kernels can overlap on the GPU (streams without ordering between them)
  *     race and give wrong results.  Calls on one stream are safe.
  *   - The scratch keeps the previous call's contents; whatever must start at
- *     zero is cleared by the call itself.
+ *     zero (the work counter, the completion counts, the bad-block marks) is
+ *     cleared by the call itself.
+ *   - The scratch used is the current device's: make the device that holds
+ *     the tensors current (cudaSetDevice) before the call.
  *   - The first call made while a device is current looks up the scratch
  *     address with a runtime call; make that first call before any stream
  *     capture starts.
@@ -359,6 +362,22 @@ ATTN_API attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out,
  * Errors: ATTN_EINVAL for a NULL or misaligned err_flag or result.
  */
 ATTN_API attn_status attn_selftest_wait_timeout(int32_t *err_flag, int32_t *result, attn_stream_t stream);
+
+/*
+ * Self-test of the exponential the bf16 prefill kernel computes on the FMA
+ * pipe for part of each score row (FlashAttention-3's "softmax under the
+ * asynchronous GEMMs" needs the exponentials to keep pace with the tensor
+ * cores: "一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解",
+ * section 二 FlashAttention-3改进).  y[i] = the kernel's 2^x[i] for
+ * i < n: a cubic in f = x - round(x) with round(x) added to the exponent,
+ * x clamped to >= -125.  The stated bound is a relative error <= 7.5e-5
+ * over [-125, 8], the kernel's range.
+ *
+ * x, y : device fp32 arrays of n elements (4-byte aligned; they may not
+ *        overlap).  Asynchronous on `stream`.
+ * Errors: ATTN_EINVAL for n < 0 or a NULL / misaligned pointer (n > 0).
+ */
+ATTN_API attn_status attn_selftest_exp2_poly(const float *x, float *y, int n, attn_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 ATTN_API const char *attn_status_str(attn_status s);
