@@ -115,21 +115,18 @@ def rotate(x, signs) -> np.ndarray:
     return (x * np.asarray(signs, dtype=np.float64)) @ hadamard(d)
 
 
-def quantize_blocks(x, block_rows: int = 128, signs=None, rotated=None):
+def quantize_blocks(x, block_rows: int = 128, signs=None):
     """Block-quantise rows of x [..., N, d] (fp32 values, e.g. bf16 inputs
     upcast) to e4m3.
 
-    ``signs`` (d values of +-1) selects incoherent processing; ``rotated``
-    may pass the rotated rows y in fp32 when the caller wants the code
-    decision taken on its own y (the rotation is a sum of d terms and its
-    fp32 rounding depends on the order of the additions).  Returns
-    (codes as float64 values on the e4m3 grid, scales float32 [..., nblk]).
+    ``signs`` (d values of +-1) selects incoherent processing: the rows are
+    rotated here, in fp64 (:func:`rotate`), and rounded to fp32 before the
+    code decision.  Returns (codes as float64 values on the e4m3 grid,
+    scales float32 [..., nblk]).
     """
     x = np.asarray(x, dtype=np.float32)
     *lead, N, d = x.shape
-    if rotated is not None:
-        y = np.asarray(rotated, dtype=np.float32)
-    elif signs is not None:
+    if signs is not None:
         y = rotate(x, signs).astype(np.float32)
     else:
         y = x
@@ -146,7 +143,7 @@ def quantize_blocks(x, block_rows: int = 128, signs=None, rotated=None):
         r = np.where(np.isinf(r), np.finfo(np.float32).max, r).astype(np.float32)
         prod = (blk * r[..., None, None]).astype(np.float32)
         codes[..., r0:r1, :] = e4m3_round(prod)
-        denom = 448.0 * np.sqrt(d) if (signs is not None or rotated is not None) else 448.0
+        denom = 448.0 * np.sqrt(d) if signs is not None else 448.0
         sc = np.where(amax == 0, 1.0, amax.astype(np.float64) / denom).astype(np.float32)
         scales[..., b] = sc
     return codes, scales

@@ -311,8 +311,25 @@ def test_merge_partials_any_split():
 
 
 def test_attention_flops():
-    assert oracle.attention_flops(4, 16, 2048, 128, True) == 4 * 4 * 16 * 128 * 2048 * 2049 // 2
-    assert oracle.attention_flops(1, 2, 128, 64, False) == 4 * 2 * 64 * 128 * 128
+    """The algorithmic FLOP count is 4*d per visible (query, key) pair (2*d for
+    q.k and 2*d for p*v).  The visible pairs are counted here two ways that do
+    not use the formula: a double loop over (i, j) with the causal rule
+    j <= i, and the nonzero entries of the oracle's materialised P on random
+    inputs.  Then the two prefill workloads hit the rounded figures printed
+    for them: 68.75 GFLOP (4 x 16 x 2048, d 128, causal) and 2.199 TFLOP
+    (1 x 32 x 16384, d 128, causal)."""
+    rng = np.random.default_rng(7)
+    for N in range(1, 10):
+        for causal in (False, True):
+            loops = sum(1 for i in range(N) for j in range(N) if (j <= i or not causal))
+            Q, K = rng.standard_normal((N, 4)), rng.standard_normal((N, 4))
+            support = int(np.count_nonzero(oracle.softmax_probs(Q, K, causal, 0.5)))
+            assert support == loops
+            for B, H, d in ((1, 1, 4), (2, 3, 64)):
+                assert oracle.attention_flops(B, H, N, d, causal) == 4 * d * B * H * loops
+    assert round(oracle.attention_flops(4, 16, 2048, 128, True) / 1e9, 2) == 68.75
+    assert round(oracle.attention_flops(1, 32, 16384, 128, True) / 1e12, 3) == 2.199
+    assert round(oracle.attention_flops(1, 2, 128, 64, False) / 1e6, 2) == 8.39
 
 
 # --------------------------------------------------------------------------
