@@ -12,6 +12,8 @@
 namespace osp {
 // One CTA waits on an mbarrier phase that never completes (selftest.cu).
 attn_status launch_wait_timeout_selftest(int32_t *err_flag, int32_t *result, cudaStream_t stream);
+// The prefill softmax's FMA-pipe 2^x on given inputs (selftest.cu).
+attn_status launch_exp2_poly_selftest(const float *x, float *y, int n, cudaStream_t stream);
 }  // namespace osp
 
 namespace {
@@ -200,6 +202,13 @@ attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_t *src_bl
 attn_status attn_selftest_wait_timeout(int32_t *err_flag, int32_t *result, attn_stream_t stream) {
     if (!err_flag || ((uintptr_t)err_flag & 3u) || ((uintptr_t)result & 3u)) return ATTN_EINVAL;
     return osp::launch_wait_timeout_selftest(err_flag, result, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_selftest_exp2_poly(const float *x, float *y, int n, attn_stream_t stream) {
+    if (n < 0) return ATTN_EINVAL;
+    if (n == 0) return ATTN_OK;
+    if (!x || !y || ((uintptr_t)x & 3u) || ((uintptr_t)y & 3u)) return ATTN_EINVAL;
+    return osp::launch_exp2_poly_selftest(x, y, n, reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_read_error(const int32_t *err_flag, int32_t *bits_out, attn_stream_t stream) {

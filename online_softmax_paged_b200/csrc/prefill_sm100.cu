@@ -40,6 +40,7 @@
 
 #include "launch.h"
 #include "ptx.cuh"
+#include "softmax_math.cuh"
 
 namespace osp {
 namespace {
@@ -152,35 +153,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
 
 // ---------------------------------------------------------------- softmax math
 
-
-// 2^x for a pair of floats on the FMA pipe, keeping the MUFU free for the
-// rest.  Range reduction x = n + f with n = round(x) (the 1.5 * 2^23 shift),
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted to 2^f on [-1/2, 1/2]
-// at Chebyshev nodes with relative-error weighting (Lawson iterations towards
-// the minimax fit; max relative error 7.5e-5 in fp32, far below the bf16
-// rounding of P); 2^n is added into the exponent field.  x is clamped to
-// >= -125 so the result stays a normal number (2^-125 ~ 0 next to l >= 1).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 0x1.fff692p-1f, c1 = 0x1.62f31ap-1f, c2 = 0x1.f0de1ap-3f, c3 = 0x1.c3f75ep-5f;
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
-    const uint64_t xc = f2_pack(x0, x1);
-    const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));           // n in the low mantissa bits
-    const uint64_t nr = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(kShift, kShift));  // -n
-    const uint64_t fr = f2_add(xc, nr);                               // f = x - n
-    uint64_t r = f2_fma(f2_pack(c3, c3), fr, f2_pack(c2, c2));
-    r = f2_fma(r, fr, f2_pack(c1, c1));
-    r = f2_fma(r, fr, f2_pack(c0, c0));
-    float p0, p1, t0, t1;
-    f2_unpack(r, p0, p1);
-    f2_unpack(t, t0, t1);
-    p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-    return f2_pack(p0, p1);
-}
 
 // Pairs k with (k % 8) >= kPolyFrom take the polynomial; the others MUFU ex2.
 constexpr int kPolyFrom = 5;  // 3 of every 8 pairs
