@@ -16,22 +16,31 @@ A step is one call of the entry point on one batch of the workload:
                        (incoherent processing on) + attn_fwd_fp8 (e4m3 QK^T, bf16 P.V)
   prefill_paged_chunked paged_attn_prefill, 8 seqs x 2048 new tokens after U{0..6144} cached,
                        32 query heads over 8 K/V heads, d=128, bs=16
-The default line reports prefill TFLOP/s and carries the paged-decode GB/s of
-decode_uniform, measured the same way in the same run, under "decode".
+The default line reports prefill_2k TFLOP/s and carries, measured the same
+way in the same run, the other workloads of the path under their own keys:
+"decode" (decode_uniform), "prefill_16k" and "decode_shared_prefix", each
+with its roofline, timing statistics, clocks, e2e and cpu_baseline.
 
 Rates use algorithmic work: prefill FLOPs = 4 * B * H * d * (visible query-key
 pairs) (causal: N(N+1)/2 per head); decode bytes = K/V bytes the sequences
 attend over (sum_s L_s * 2 * H * d * 2; for the shared-prefix workload the
 unique physical bytes, logical bytes reported beside).
 
-Timing: W untimed warm-up steps, then the K steps captured once in a CUDA
-graph and replayed between barrier + cuda.synchronize, CUDA events on the
-launching stream around the replay (device time of K back-to-back steps;
---eager times K separate calls with events around each instead);
-inputs rotate over copies whose total exceeds L2 (prefill) or exceed it alone
-(decode pools of GB).  Multi-GPU (torchrun): every rank runs its own replica
-(independent problems, weak scaling, no collective on the data path); the
-time is the max over ranks.  Only rank 0 prints the JSON line.
+Timing: W untimed warm-up steps; the K steps are captured once in a CUDA
+graph; after an untimed soak the graph is replayed back to back, each replay
+(exactly K steps) between its own CUDA events on the launching stream, until
+the timed region lasts at least --region-s seconds (1 s), the region
+bracketed by barrier + cuda.synchronize.  value = work of all timed steps /
+region time; timing_stats gives the median per-step time over the replays
+and its spread; the clocks are the nvidia-smi samples taken inside the
+region.  The roofline divides the dominant kernel's mean launch time into
+its algorithmic work, against the measured burst peak (tensor-bound) or the
+measured copy bandwidth (HBM-bound).  --eager times K separate calls
+instead.  Inputs rotate over copies whose total exceeds L2 (prefill) or
+exceed it alone (decode pools of GB).  Multi-GPU (torchrun): every rank runs
+its own replica (independent problems, weak scaling, no collective on the
+data path); the time is the max over ranks.  Only rank 0 prints the JSON
+line.
 """
 from __future__ import annotations
 
@@ -169,7 +178,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-KERNEL_SOURCES = {"prefill_bf16_kernel": ("prefill_sm100.cu", "ptx.cuh", "launch.h"),
+KERNEL_SOURCES = {"prefill_bf16_kernel": ("prefill_sm100.cu", "softmax_math.cuh", "ptx.cuh", "launch.h"),
                   "decode_split_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h"),
                   "decode_mma_kernel": ("decode_paged.cu", "ptx.cuh", "launch.h"),
                   "kv_append_kernel": ("kv_cache_ops.cu", "ptx.cuh", "launch.h"),
@@ -318,6 +327,12 @@ class Decode:
             q = torch.randn((base.num_seqs, 32, base.d), generator=g, device=device).to(torch.bfloat16)
             self.p = W.PagedInputs(q, base.k_cache, base.v_cache, base.block_table, base.seq_lens,
                                    base.block_size, base.scale)
+        elif name == "decode_shared_prefix_small":
+            # 48 sequences (6 groups) of the shared-prefix workload in a
+            # 4000-block pool (2.1 GB of K/V, above L2): the case profiler
+            # captures run on
+            self.p = W.paged_shared_prefix(device=device, seed=seed, **{**W.DECODE_SHARED_PREFIX, "num_seqs": 48,
+                                                                         "pool": 4000})
         elif name == "decode_uniform_small":
             # 16 sequences of the uniform workload in a 4000-block pool (1 GiB
             # of K/V, still above L2): the case profiler captures run on
@@ -330,7 +345,7 @@ class Decode:
                            self.p.block_table, self.p.seq_lens, self.p.block_size, self.p.scale)
         self.logical = W.logical_kv_bytes(kv)   # K/V bytes of the key/value heads attended
         self.unique = W.unique_kv_bytes(kv)
-        self.work = float(self.unique if name == "decode_shared_prefix" else self.logical)  # bytes per step
+        self.work = float(self.unique if name.startswith("decode_shared_prefix") else self.logical)  # bytes per step
         self.O = torch.empty_like(self.p.q)
         self.LSE = torch.empty(self.p.q.shape[:2], dtype=torch.float32, device=device)
         import online_softmax_paged_b200 as osp
@@ -795,7 +810,8 @@ def make_workload(name, device, seed=0):
         return Prefill(W.PREFILL_CAUSAL_2K, name, device, seed)
     if name == "prefill_16k":
         return Prefill(W.PREFILL_CAUSAL_16K, name, device, seed)
-    if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small", "decode_gqa_g4", "decode_gqa_g8"):
+    if name in ("decode_uniform", "decode_shared_prefix", "decode_uniform_small", "decode_shared_prefix_small",
+                "decode_gqa_g4", "decode_gqa_g8"):
         return Decode(name, device, seed)
     if name == "kv_append":
         return KVAppend(name, device, seed)
@@ -812,13 +828,34 @@ def make_workload(name, device, seed=0):
 
 # ---------------------------------------------------------------- timing
 
-def time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s=0.0):
-    """The K timed steps captured once into a CUDA graph and replayed between
-    barrier + synchronize, CUDA events around the replay: device time of K
-    back-to-back steps, without the host's per-call launch cost (a serving
-    loop replays its decode steps the same way).  Steps of several launches
-    whose roofline is one kernel's also get a graph of that kernel alone.
-    Returns (per-step or per-kernel ms list, total ms, wall s)."""
+def _region(graph, replays, st, device, ws):
+    """``replays`` back-to-back replays of ``graph`` between barrier +
+    synchronize on both sides, a pair of CUDA events around each on the
+    launching stream.  Returns (per-replay ms, total ms from the first start
+    event to the last end event, (t0, t1) perf_counter span)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    barrier(ws)
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    for a, b in evs:
+        a.record(st)
+        graph.replay()
+        b.record(st)
+    torch.cuda.synchronize(device)
+    barrier(ws)
+    t1 = time.perf_counter()
+    return [a.elapsed_time(b) for a, b in evs], evs[0][0].elapsed_time(evs[-1][1]), (t0, t1)
+
+
+def time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s=0.0, region_s=1.0):
+    """The K timed steps captured once into a CUDA graph; the graph is
+    replayed back to back, each replay (exactly K steps) between its own
+    CUDA events, until the timed region lasts at least ``region_s`` seconds
+    (every rank replays the same number of times).  Device time only, without
+    the host's per-call launch cost (a serving loop replays its decode steps
+    the same way).  Steps of several launches whose roofline is one kernel's
+    also get a graph of that kernel alone, timed the same way after the
+    region.  Returns a dict of the timings."""
     st = torch.cuda.current_stream(device)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -830,54 +867,42 @@ def time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s=0.0):
         with torch.cuda.graph(gk):
             for i in range(steps):
                 wl.dominant(warmup + i, osp)
-    g.replay()  # first replay uploads the graph
+    g.replay()  # the first replay uploads the graph
     if gk is not None:
         gk.replay()
     torch.cuda.synchronize(device)
-    # the soak replays the same graph right before the timed replay, so the
-    # timed steps run at the clocks a loaded GPU settles to (capturing left
-    # the GPU idle)
+    # one replay sizes the region
+    one_ms = _region(g, 1, st, device, 1)[1]
+    replays = max(3, math.ceil(region_s * 1e3 / max(one_ms, 1e-3))) if region_s > 0 else 1
+    replays = int(max_over_ranks(float(replays), ws))
+    # the soak replays the same graph right before the timed region, so the
+    # region starts at the clocks a loaded GPU settles to (capturing left the
+    # GPU idle)
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < soak_s:
         g.replay()
         torch.cuda.synchronize(device)
-    barrier(ws)
-    torch.cuda.synchronize(device)
-    t_region0 = time.perf_counter()
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    g0.record(st)
-    g.replay()
-    g1.record(st)
-    torch.cuda.synchronize(device)
-    barrier(ws)
-    wall = time.perf_counter() - t_region0
-    total_ms = g0.elapsed_time(g1)
-    per = [total_ms / steps] * steps
+    rep, total_ms, span = _region(g, replays, st, device, ws)
+    out = {"rep_ms": rep, "total_ms": total_ms, "span": span, "replays": replays, "steps": steps,
+           "kernel_rep_ms": None, "timing": "graph"}
     if gk is not None:
-        k0 = torch.cuda.Event(enable_timing=True)
-        k1 = torch.cuda.Event(enable_timing=True)
-        k0.record(st)
-        gk.replay()
-        k1.record(st)
-        torch.cuda.synchronize(device)
-        per = [k0.elapsed_time(k1) / steps] * steps
+        out["kernel_rep_ms"] = _region(gk, replays, st, device, ws)[0]
     del g, gk
-    return per, total_ms, wall
+    return out
 
 
-def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0, graph=False):
-    """W warm-up steps, an optional untimed soak (so the clocks sampled
-    around the timed region reflect a loaded GPU), then K timed steps between
-    barrier + synchronize with CUDA events around every launch (or, with
-    ``graph``, around one replay of the K steps captured in a CUDA graph)."""
+def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0, graph=False, region_s=1.0):
+    """W warm-up steps, then the timed region: with ``graph``, replays of the
+    K steps captured in a CUDA graph (time_steps_graph); otherwise K eager
+    calls with CUDA events around every launch, after an optional untimed
+    soak.  Returns a dict of the timings."""
     st = torch.cuda.current_stream(device)
     for i in range(warmup):
         wl.step(i, osp)
     torch.cuda.synchronize(device)
     if graph:
         try:
-            return time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s) + ("graph",)
+            return time_steps_graph(wl, osp, steps, warmup, device, ws, soak_s, region_s)
         except Exception as e:  # capture unsupported here: time eagerly
             print(f"CUDA graph capture failed ({e!r}); timing eagerly", file=sys.stderr)
             torch.cuda.synchronize(device)
@@ -905,47 +930,121 @@ def time_steps(wl, osp, steps, warmup, device, ws, soak_s=0.0, graph=False):
     g1.record(st)
     torch.cuda.synchronize(device)
     barrier(ws)
-    wall = time.perf_counter() - t_region0
+    span = (t_region0, time.perf_counter())
     per = [a.elapsed_time(b) for a, b in evs]
+    kper = None
     if hasattr(wl, "kernel_events"):
         wl.record = False
-        per = [a.elapsed_time(b) for a, b in wl.kernel_events]
-    total_ms = g0.elapsed_time(g1)
-    return per, total_ms, wall, "eager"
+        kper = [a.elapsed_time(b) for a, b in wl.kernel_events]
+    # eager: every step is its own "replay" of one step
+    return {"rep_ms": per, "total_ms": g0.elapsed_time(g1), "span": span, "replays": steps, "steps": 1,
+            "kernel_rep_ms": kper, "timing": "eager"}
 
 
-def roofline(wl, per_ms, pk, pk_src, bound, clocks=None):
-    """Roofline of the dominant kernel from its mean launch time.  Tensor-bound
-    kernels are compared with the measured burst bf16 peak, or with the
-    measured sustained (power-capped) peak when the clocks sampled around
-    the timed region show the power cap holding the SM clock down."""
-    launch_ms = statistics.mean(per_ms)
+def timing_stats(tm):
+    """Per-step statistics of a timed region: the median per-replay time over
+    K, its spread, and the mean over the whole region."""
+    per = sorted(r / tm["steps"] for r in tm["rep_ms"])
+    n = len(per)
+
+    def q(f):
+        return per[min(n - 1, max(0, int(round(f * (n - 1)))))]
+
+    med = statistics.median(per)
+    return {"replays": tm["replays"], "steps_per_replay": tm["steps"], "steps_timed": tm["replays"] * tm["steps"],
+            "region_s": round(tm["span"][1] - tm["span"][0], 3), "timing": tm["timing"],
+            "per_step_ms": {"median": round(med, 5), "mean": round(tm["total_ms"] / (tm["replays"] * tm["steps"]), 5),
+                            "min": round(per[0], 5), "p10": round(q(0.1), 5), "p90": round(q(0.9), 5),
+                            "max": round(per[-1], 5)},
+            "spread_p10_p90_pct": round(100.0 * (q(0.9) - q(0.1)) / med, 2) if med > 0 else None}
+
+
+def roofline(wl, launch_ms, pk, pk_src, bound, clocks=None):
+    """Roofline of the dominant kernel from its mean launch time over the
+    timed region.  Tensor-bound kernels are compared with the measured burst
+    bf16 peak (one fixed denominator, whatever the clocks did); the fraction
+    of the measured sustained (power-capped) peak is reported beside it with
+    the median SM clock of the region."""
     achieved = wl.work / (launch_ms * 1e-3) / wl.scale_unit
     extra = {}
     if bound == "tensor":
         burst = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         sustained = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        capped = bool(clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
-                      and "sw_power_cap" in clocks.get("reasons", [])
-                      and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
         f = getattr(wl, "peak_factor", 1.0)  # FP8 QK^T: the blended e4m3 / bf16 peak
         burst, sustained = burst * f, sustained * f
-        peak = sustained if capped else burst
-        extra = {"peak_kind": "sustained (power-capped clocks in the timed window)" if capped else "burst",
-                 "frac_of_burst": round(achieved / burst, 4), "frac_of_sustained": round(achieved / sustained, 4)}
+        peak = burst
+        extra = {"peak_kind": "burst bf16 (measured cuBLAS-class matmul)",
+                 "frac_of_sustained": round(achieved / sustained, 4), "peak_sustained": round(sustained, 1)}
+        if clocks and clocks.get("sm_mhz"):
+            extra["sm_mhz_median_in_region"] = clocks["sm_mhz"]
         if f != 1.0:
             extra["peak_kind"] += "; bf16 peak x 4/3 (QK^T at the e4m3 rate, P.V at the bf16 rate)"
         unit = "TFLOP/s"
     else:
         peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         unit = "GB/s"
-        extra = {"peak_kind": "copy bandwidth"}
+        extra = {"peak_kind": "copy bandwidth (measured)"}
     spec = SPEC_PEAKS["bf16_tflops"] * getattr(wl, "peak_factor", 1.0) if bound == "tensor" else SPEC_PEAKS["hbm_gbs"]
     extra["frac_of_spec"] = round(achieved / spec, 4)
     tr = recorded_traffic(wl.kernel, wl.name)
     return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": tr, "peak_source": pk_src,
-            "kernel": wl.kernel, "launch_ms": round(launch_ms, 5), **extra}
+            "kernel": wl.kernel, "launch_ms": round(launch_ms, 5), "work_per_launch": wl.work, **extra}
+
+
+BAD_CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def measure(wl, osp, args, device, ws, clocks, pk, pk_src, region_s):
+    """Time one workload (its timed region re-measured once if the clocks
+    sampled inside it show a hardware or thermal slowdown) and return its
+    rate, roofline, statistics and clocks."""
+    bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill, Fp8Prefill)) else "hbm"
+    remeasured = False
+    for attempt in range(2):
+        tm = time_steps(wl, osp, args.steps, args.warmup if attempt == 0 else 1, device, ws, soak_s=args.soak,
+                        graph=not args.eager, region_s=region_s)
+        clk = clocks.summary(*tm["span"])
+        if not set(clk["reasons"]) & set(BAD_CLOCK_REASONS) or attempt == 1:
+            break
+        remeasured = True
+    n_steps = tm["replays"] * tm["steps"]
+    t_max = max_over_ranks(tm["total_ms"], ws)
+    work_all = sum_over_ranks(wl.work * n_steps, ws)
+    value = work_all / (t_max * 1e-3) / wl.scale_unit
+    ms_step = t_max / n_steps
+    if tm["kernel_rep_ms"] is not None:  # the dominant kernel timed on its own
+        kn = len(tm["kernel_rep_ms"]) * tm["steps"] if tm["timing"] == "graph" else len(tm["kernel_rep_ms"])
+        launch_ms = max_over_ranks(sum(tm["kernel_rep_ms"]) / kn, ws)
+    else:
+        launch_ms = ms_step  # one launch, or a call whose kernels the events wrap together
+    stats = timing_stats(tm)
+    if clk.get("sm_mhz"):
+        stats["kcycles_per_step_at_median_mhz"] = round(ms_step * clk["sm_mhz"], 2)
+    clk = {**clk, "window": "timed region only", "remeasured": remeasured,
+           "rejected": bool(set(clk["reasons"]) & set(BAD_CLOCK_REASONS))}
+    return {"value": value, "ms_per_step": ms_step, "steps_timed": n_steps, "timing": tm["timing"],
+            "roofline": roofline(wl, launch_ms, pk, pk_src, bound, clk), "stats": stats, "clocks": clk,
+            "gpu_launches": wl.launches_per_step * n_steps}
+
+
+def cpu_leg(wl, budget_s):
+    work, dt, sample = wl.cpu_sample(budget_s)
+    return {"value": round(work / dt / wl.scale_unit, 6), "unit": wl.unit, "cores": _cpu_threads(),
+            "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+
+
+def e2e_leg(wl, osp, steps, device, ws):
+    e2e_ms, h2d, d2h = wl.e2e(osp, steps, device)
+    e2e_ms = max_over_ranks(e2e_ms, ws)
+    val = sum_over_ranks(wl.work, ws) / (e2e_ms * 1e-3) / wl.scale_unit
+    return {"value": round(val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(e2e_ms, 5)}
+
+
+# the other workloads the default line carries, measured the same way in the
+# same run: the long causal prefill and the two paged-decode workloads
+DEFAULT_LEGS = ("decode_uniform", "prefill_16k", "decode_shared_prefix")
 
 
 def run_ours(args):
@@ -959,55 +1058,43 @@ def run_ours(args):
     import online_softmax_paged_b200 as osp
     osp.load()
     pk, pk_src = peaks()
+    e2e_steps = max(3, min(args.steps, 20))
 
     wl = make_workload(args.workload, device, seed=args.seed + rank)
-    bound = "tensor" if isinstance(wl, (Prefill, PagedPrefill, Fp8Prefill)) else "hbm"
     with ClockSampler(local) as clocks:
-        t_load0 = time.perf_counter()
-        per, total_ms, wall, timing = time_steps(wl, osp, args.steps, args.warmup, device, ws, soak_s=args.soak,
-                                                 graph=not args.eager)
-        t_load1 = time.perf_counter()
-    t_max = max_over_ranks(total_ms, ws)
-    work_all = sum_over_ranks(wl.work * args.steps, ws)
-    value = work_all / (t_max * 1e-3) / wl.scale_unit
-    clk = clocks.summary(t_load0, t_load1)
-    rl = roofline(wl, per, pk, pk_src, bound, clk)
-
-    e2e_ms, h2d, d2h = wl.e2e(osp, max(3, min(args.steps, 20)), device)
-    e2e_ms = max_over_ranks(e2e_ms, ws)
-    e2e_val = sum_over_ranks(wl.work, ws) / (e2e_ms * 1e-3) / wl.scale_unit
-
-    extra = {}
-    if args.workload == "prefill_2k" and not args.no_decode:
-        dec = make_workload("decode_uniform", device, seed=args.seed + rank)
-        per_d, total_d, _, timing_d = time_steps(dec, osp, args.steps, args.warmup, device, ws,
-                                                 soak_s=min(args.soak, 0.5), graph=not args.eager)
-        td = max_over_ranks(total_d, ws)
-        extra["decode"] = {"workload": "decode_uniform", "value": round(sum_over_ranks(dec.work * args.steps, ws)
-                                                                        / (td * 1e-3) / 1e9, 2),
-                           "unit": "GB/s", "ms_per_step": round(td / args.steps, 5),
-                           "roofline": roofline(dec, per_d, pk, pk_src, "hbm"),
-                           "config": {**dec.config(), "timing": timing_d},
-                           "gpu_launches": dec.launches_per_step * args.steps}
-        del dec
-
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu:
-        work, dt, sample = wl.cpu_sample(args.cpu_budget)
-        cpu = {"value": round(work / dt / wl.scale_unit, 6), "unit": wl.unit, "cores": _cpu_threads(),
-               "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+        m = measure(wl, osp, args, device, ws, clocks, pk, pk_src, args.region_s)
+        e2e = e2e_leg(wl, osp, e2e_steps, device, ws)
+        cpu = cpu_leg(wl, args.cpu_budget) if rank == 0 and ws == 1 and not args.no_cpu else None
+        config = wl.config()
+        del wl
+        legs = {}
+        if args.workload == "prefill_2k" and not args.no_decode:
+            for name in DEFAULT_LEGS:
+                torch.cuda.empty_cache()
+                lw = make_workload(name, device, seed=args.seed + rank)
+                lm = measure(lw, osp, args, device, ws, clocks, pk, pk_src, args.region_s)
+                leg = {"workload": name, "value": round(lm["value"], 3), "unit": lw.unit,
+                       "ms_per_step": round(lm["ms_per_step"], 5), "steps": args.steps,
+                       "roofline": lm["roofline"], "timing_stats": lm["stats"], "clocks": lm["clocks"],
+                       "e2e": e2e_leg(lw, osp, min(e2e_steps, 5), device, ws),
+                       "cpu_baseline": (cpu_leg(lw, args.cpu_budget) if rank == 0 and ws == 1 and not args.no_cpu
+                                        else None),
+                       "config": {**lw.config(), "timing": lm["timing"]}, "gpu_launches": lm["gpu_launches"]}
+                legs[name] = leg
+                del lw
+        # the first leg keeps its historical key
+        extra = {("decode" if k == "decode_uniform" else k): v for k, v in legs.items()}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": ws, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16" if isinstance(wl, Fp8Prefill) else "bf16",
+        line = {"metric": METRIC, "value": round(m["value"], 3), "unit": m["roofline"]["unit"], "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(m["ms_per_step"], 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3+bf16" if args.workload.startswith("prefill_fp8") else "bf16",
                 "data": "synthetic (seeded N(0,1), bf16)",
-                "config": {**wl.config(), "parallelism": f"replicas{ws}" if ws > 1 else "single", "timing": timing},
-                "roofline": rl, "cpu_baseline": cpu,
-                "e2e": {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-                "gpu_launches": wl.launches_per_step * args.steps, "clocks": clk,
-                "timed_wall_s": round(wall, 3), **extra}
+                "config": {**config, "parallelism": f"replicas{ws}" if ws > 1 else "single", "timing": m["timing"]},
+                "roofline": m["roofline"], "timing_stats": m["stats"], "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+                "timed_wall_s": m["stats"]["region_s"], **extra}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
@@ -1137,12 +1224,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_2k",
                     choices=["prefill_2k", "prefill_16k", "decode_uniform", "decode_shared_prefix",
-                             "decode_uniform_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8",
+                             "decode_uniform_small", "decode_shared_prefix_small", "kv_append", "block_copy", "decode_gqa_g4", "decode_gqa_g8",
                              "prefill_paged_chunked", "prefill_fp8_2k", "prefill_fp8_16k"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode leg of the default line")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the extra legs of the default line (decode_uniform, prefill_16k, decode_shared_prefix)")
+    ap.add_argument("--region-s", type=float, default=1.0,
+                    help="minimum length of each timed region: the K-step graph is replayed until it lasts this "
+                         "long (0: one replay)")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing (clocks)")
     ap.add_argument("--eager", action="store_true",
                     help="time K eager calls instead of one replay of the K steps captured in a CUDA graph")
