@@ -91,6 +91,7 @@ struct DecodeArgs {
     int bs_shift;         // log2(block_size)
     float scale_log2;     // scale * log2(e)
     int fused_plan;       // grouped kernel: every CTA computes the plan itself (no plan kernel)
+    int sched_w;          // grouped kernel: schedule width (math warps of the launch, at most kMaxWorkers)
 };
 
 __device__ __forceinline__ bool seq_len_ok(int L, const DecodeArgs &a) {
@@ -537,16 +538,18 @@ __global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(D
 //
 // Work is not taken from a queue: every (sequence, key/value head) row has
 // ceil(L / 16) tiles, the rows are laid end to end (sequence-major), and
-// worker w of kWorkers takes tiles [w c, (w + 1) c) of that line, with
-// c = max(ceil(T / kWorkers), kMinTiles) for T tiles in all.  Every worker
-// then streams the same number of bytes (the last one fewer), whatever the
-// length mix; a worker's run crosses row boundaries as it comes.  A row cut
-// by worker boundaries into n segments gets n partials, stored at slots
-// worker + row (so one row's slots are consecutive, and all slots fit in
-// kWorkers + rows), and is merged by the worker that completes its last
-// segment.  The plan depends on the lengths and sizes only (kWorkers is a
-// constant, not the GPU's warp count), so results do not depend on the
-// physical block ids or on which warp ran a worker.
+// worker w of nw takes tiles [floor(w T / nw), floor((w + 1) T / nw)) of
+// that line for T tiles in all, with nw = min(W, max(1, floor(T / 8))) and
+// W the launch's math warps (at most kMaxWorkers): every warp has a run,
+// the runs differ by at most one tile, and none is shorter than 8 tiles
+// (128 keys) unless T is.  Every worker then streams the same number of
+// bytes whatever the length mix; a worker's run crosses row boundaries as
+// it comes.  The worker holding tile x is floor(((x + 1) nw - 1) / T).  A
+// row cut by worker boundaries into n segments gets n partials, stored at
+// slots worker + row (so one row's slots are consecutive, and all slots fit
+// in nw + rows), merged by decode_merge_kernel.  The plan depends on the
+// lengths, the sizes and the launch's width only, so results do not depend
+// on the physical block ids or on which warp ran a worker.
 //
 // A CTA is 8 math warps and one producer warp (in a warpgroup of its own,
 // the register split moving registers to the math warps).  Lane c of the
@@ -558,8 +561,7 @@ __global__ void __launch_bounds__(Warps<G>::value * 32, 1) decode_split_kernel(D
 constexpr int kCons = 8;                          // math warps per CTA
 constexpr int kMmaThreads = (kCons + 4) * 32;     // + the producer's warpgroup
 constexpr int kConsRegs = 224, kProdRegs = 56;    // 256 x 224 + 128 x 56 = 384 x 168
-constexpr int kWorkers = 148 * kCons;             // schedule width: one worker per math warp of 148 SMs
-constexpr int kMaxWorkers = 148 * 10;             // workspace bound (at least kWorkers)
+constexpr int kMaxWorkers = 148 * 10;             // schedule width bound (the workspace holds its slots)
 constexpr int kMinTiles = 8;                      // shortest worker run: 128 keys
 constexpr float kLazyLog2 = 8.f;  // rescale only when the max grows by more than 2^8
 constexpr int kScratchBytes = 8 * kD * 4;  // per math warp: up to 8 unnormalised O rows (fp32)
@@ -645,20 +647,37 @@ __device__ __forceinline__ int seq_of_tile(const DecodeArgs &a, const int32_t *s
     return lo;
 }
 
+// The schedule: T tiles over nw workers in runs differing by at most one
+// tile.
+struct Sched {
+    long long T, nw;
+};
+
+__host__ __device__ __forceinline__ long long sched_nw(long long T, int W) {
+    const long long by_len = T / kMinTiles;
+    return by_len < 1 ? 1 : (by_len < W ? by_len : W);
+}
+
+// first tile of worker w's run (w in [0, nw]; w = nw gives T)
+__device__ __forceinline__ long long run_begin(const Sched &sc, long long w) { return w * sc.T / sc.nw; }
+
+// the worker whose run holds tile x (x in [0, T))
+__device__ __forceinline__ long long worker_of(const Sched &sc, long long x) { return ((x + 1) * sc.nw - 1) / sc.T; }
+
 // Start worker run ps.w + stride (false: none left).
-__device__ __forceinline__ bool next_worker(SchedPos &ps, long long T, int chunk, long long nw, int stride) {
+__device__ __forceinline__ bool next_worker(SchedPos &ps, const Sched &sc, int stride) {
     ps.w += stride;
-    if (ps.w >= nw) return false;
-    ps.x_begin = ps.x = (long long)ps.w * chunk;
-    ps.x_end = min(T, ps.x + chunk);
+    if (ps.w >= sc.nw) return false;
+    ps.x_begin = ps.x = run_begin(sc, ps.w);
+    ps.x_end = run_begin(sc, ps.w + 1);
     return true;
 }
 
 // The next item of a math warp (warp-uniform): the rest of the current row
 // inside the current worker's run, then the next worker (w + stride).
-__device__ __forceinline__ void next_seg_item(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
-                                              long long nw, int stride, int &s_hint, SchedPos &ps, SegItem &it) {
-    if (ps.x >= ps.x_end && !next_worker(ps, T, chunk, nw, stride)) {
+__device__ __forceinline__ void next_seg_item(const DecodeArgs &a, const int32_t *starts, const Sched &sc, int stride,
+                                              int &s_hint, SchedPos &ps, SegItem &it) {
+    if (ps.x >= ps.x_end && !next_worker(ps, sc, stride)) {
         it.nt = 0;
         return;
     }
@@ -703,11 +722,11 @@ __device__ __forceinline__ int walk_block_id(const DecodeArgs &a, const TileWalk
 }
 
 // Step to the next tile (false: the math warp's schedule is done).
-__device__ __forceinline__ bool walk_advance(const DecodeArgs &a, const int32_t *starts, long long T, int chunk,
-                                             long long nw, int stride, TileWalk &wk) {
+__device__ __forceinline__ bool walk_advance(const DecodeArgs &a, const int32_t *starts, const Sched &sc, int stride,
+                                             TileWalk &wk) {
     ++wk.ps.x;
     if (wk.ps.x >= wk.ps.x_end) {
-        if (!next_worker(wk.ps, T, chunk, nw, stride)) return false;
+        if (!next_worker(wk.ps, sc, stride)) return false;
         walk_locate(a, starts, wk);
         return true;
     }
@@ -728,15 +747,15 @@ __device__ __forceinline__ bool walk_advance(const DecodeArgs &a, const int32_t 
 // fp32), row g's max / sum in lane 4g.  A row in one segment is written
 // directly; otherwise the partial goes to its slot for decode_merge_kernel.
 template <int G>
-__device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &it, const int32_t *starts, int chunk,
-                                           int lane, float *scratch, float m, float l, bool saw_bad) {
+__device__ __forceinline__ void finish_seg(const DecodeArgs &a, const SegItem &it, const int32_t *starts,
+                                           const Sched &sc, int lane, float *scratch, float m, float l, bool saw_bad) {
     const int s = it.s;
     // the row's place in the schedule: its tiles [row_begin, row_begin + nts)
-    // span workers row_begin / chunk .. (row_begin + nts - 1) / chunk
+    // span workers worker_of(row_begin) .. worker_of(row_begin + nts - 1)
     const int nts = starts[s + 1] - starts[s];
     const long long row_begin = (long long)a.Hkv * starts[s] + (long long)it.h * nts;
     const int r = s * a.Hkv + it.h;
-    const int nsplit = (int)((row_begin + nts - 1) / chunk - row_begin / chunk) + 1;
+    const int nsplit = (int)(worker_of(sc, row_begin + nts - 1) - worker_of(sc, row_begin)) + 1;
     const int slot = it.w + r;
     const size_t sh0 = (size_t)s * a.H + (size_t)it.h * G;
     const int gl = lane & 7;  // lanes 0..G-1: the row they report
@@ -839,10 +858,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         starts = st;
     }
     __syncthreads();  // barriers initialised, offsets staged
-    // the schedule: T tiles in all, runs of `chunk` tiles, nw workers with work
-    const long long T = (long long)starts[a.num_seqs] * a.Hkv;
-    const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
-    const long long nw = (T + chunk - 1) / chunk;
+    // the schedule: T tiles in all over nw workers
+    Sched sc;
+    sc.T = (long long)starts[a.num_seqs] * a.Hkv;
+    sc.nw = sched_nw(sc.T, a.sched_w);
     const int stride = gridDim.x * kCons;
 
     if (wid >= kCons) {
@@ -854,7 +873,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         wk.ps.w = blockIdx.x * kCons + c - stride;
         wk.ps.x = wk.ps.x_end = 0;
         wk.s = 0;
-        wk.live = c < kCons && next_worker(wk.ps, T, chunk, nw, stride);
+        wk.live = c < kCons && sc.T > 0 && next_worker(wk.ps, sc, stride);
         if (wk.live) {
             walk_locate(a, starts, wk);
             wk.id = walk_block_id(a, wk);
@@ -888,7 +907,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                         tma_load_2d(dst + kTileBytes + 2048, &tmV, fb, 64, y);
                     }
                     ++gi;
-                    wk.live = walk_advance(a, starts, T, chunk, nw, stride, wk);
+                    wk.live = walk_advance(a, starts, sc, stride, wk);
                     if (wk.live) wk.id = walk_block_id(a, wk);  // consumed at the next issue
                     t_last = globaltimer_ns();
                 }
@@ -935,7 +954,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     }
     for (;;) {
         SegItem cur;
-        next_seg_item(a, starts, T, chunk, nw, stride, s_hint, ps, cur);
+        if (sc.T == 0) break;
+        next_seg_item(a, starts, sc, stride, s_hint, ps, cur);
         if (cur.nt == 0) break;
         // Q fragments of the group (rows gq < G; 16-dim k-steps): a0 = dims
         // 16ks + 2tq, +1 and a2 = dims 16ks + 8 + 2tq, +1 of query head gq
@@ -1069,7 +1089,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             }
         }
         __syncwarp();
-        finish_seg<G>(a, cur, starts, chunk, lane, scratch, m, lt, saw_bad);
+        finish_seg<G>(a, cur, starts, sc, lane, scratch, m, lt, saw_bad);
         __syncwarp();  // scratch reads done before the next segment writes it
     }
 }
@@ -1095,11 +1115,12 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) 
     const int st0 = __ldcg(starts + s), st1 = __ldcg(starts + s + 1), stn = __ldcg(starts + a.num_seqs);
     const int nts = st1 - st0;
     if (nts == 0) return;  // empty or invalid length: written with the plan
-    const long long T = (long long)stn * a.Hkv;
-    const int chunk = (int)max((T + kWorkers - 1) / kWorkers, (long long)kMinTiles);
+    Sched sc;
+    sc.T = (long long)stn * a.Hkv;
+    sc.nw = sched_nw(sc.T, a.sched_w);
     const long long row_begin = (long long)a.Hkv * st0 + (long long)h * nts;
-    const int w0 = (int)(row_begin / chunk);
-    const int nsplit = (int)((row_begin + nts - 1) / chunk) - w0 + 1;
+    const int w0 = (int)worker_of(sc, row_begin);
+    const int nsplit = (int)worker_of(sc, row_begin + nts - 1) - w0 + 1;
     if (nsplit == 1) return;  // written by its segment
     const size_t slot0 = (size_t)w0 + (size_t)s * a.Hkv + h;
     const float *plse = a.part_lse + slot0 * G + g;                                      // partial q at plse[q G]
@@ -1258,20 +1279,24 @@ attn_status launch_mma(const DecodeArgs &a, const DecodeLaunch &p, int dev, int 
     cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(kMmaThreads);
     cfg.dynamicSmemBytes = kMmaSmem;
+    // the schedule's width: every math warp of the launch (the workspace holds
+    // the slots of at most kMaxWorkers)
+    DecodeArgs am = a;
+    am.sched_w = sms * kCons < kMaxWorkers ? sms * kCons : kMaxWorkers;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_mma_kernel<G>, tk, tv, a) != cudaSuccess) return ATTN_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_mma_kernel<G>, tk, tv, am) != cudaSuccess) return ATTN_ECUDA;
     // the rows left in partials, merged by a programmatic dependent
     const long long rows_q = (long long)a.num_seqs * a.H;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3((unsigned)((rows_q + 7) / 8));
     mcfg.blockDim = dim3(256);
     mcfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&mcfg, decode_merge_kernel, a, G) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+    return cudaLaunchKernelEx(&mcfg, decode_merge_kernel, am, G) == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
 attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
@@ -1331,6 +1356,7 @@ attn_status launch_paged_decode(const DecodeLaunch &p, cudaStream_t stream) {
 
     // the grouped kernel plans in every CTA when the offsets fit in shared memory
     a.fused_plan = sched && p.num_seqs <= kMaxSmemSeqs ? 1 : 0;
+    a.sched_w = 0;  // set by launch_mma
     if (!a.fused_plan) {
         decode_plan_kernel<<<1, 1024, 0, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
