@@ -25,6 +25,8 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the
  *     library allocates no device memory and keeps no pointer after return.
+ *     (paged_cow_plan, the host half of copy-on-write, is the exception: it
+ *     edits HOST arrays and makes no device call.)
  *   - Calls are asynchronous on `stream` (0 = legacy default stream); nothing
  *     synchronises the host.  Outputs are valid once the stream reaches the
  *     launch.
@@ -62,7 +64,8 @@ typedef enum {
     ATTN_EINVAL = 1,       /* bad pointer, size, alignment or shape */
     ATTN_EUNSUPPORTED = 2, /* valid but not implemented (head dim, dtype) */
     ATTN_ECUDA = 3,        /* a CUDA runtime / driver call failed */
-    ATTN_EDEVICE = 4       /* the device reported a problem via err_flag */
+    ATTN_EDEVICE = 4,      /* the device reported a problem via err_flag */
+    ATTN_ENOBLOCKS = 5     /* paged_cow_plan: the free list ran out */
 } attn_status;
 
 typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
@@ -342,6 +345,43 @@ ATTN_API attn_status paged_kv_append(const void *k_new, const void *v_new, const
 ATTN_API attn_status paged_block_copy(void *k_cache, void *v_cache, const int32_t *src_blocks,
                                       const int32_t *dst_blocks, int num_pairs, int num_blocks, int H, int d,
                                       int block_size, attn_dtype dt, int32_t *err_flag, attn_stream_t stream);
+
+/*
+ * Copy-on-write planning on the host: the table and reference-count half of
+ * copying a shared block before a sequence writes into it
+ * ("一文掌握大模型推理加速：FlashAttention与PagedAttention技术详解", section 三
+ * 内存共享机制: shared blocks carry a reference count; a write to a block
+ * whose count is above 1 first copies it to a free block, the writer's table
+ * entry is redirected to the copy and the counts are adjusted; the other
+ * sharers keep the old contents).  The copies it plans are then made on the
+ * device by paged_block_copy, before the writes (paged_kv_append).
+ *
+ * All arrays are HOST memory owned by the caller; nothing is allocated and
+ * no device call is made.
+ * block_table  : int32 [num_seqs, max_blocks_per_seq], edited in place:
+ *                the entries of copied blocks point at their copies.
+ * ref_counts   : int32 [num_blocks], edited in place (sharers per block).
+ * free_list    : int32 [*free_count], a stack of free block ids (count 0):
+ *                copies take blocks from its end; *free_count is updated.
+ * write_seqs,
+ * write_blocks : int32 [num_writes]: the pending writes, (sequence, logical
+ *                block), in the order they happen.  A write whose block has
+ *                count 1 is the writer's own (no copy); a repeated write, or
+ *                the last sharer's write, finds its block exclusive.
+ * src_out,
+ * dst_out      : int32 [num_writes] (capacity): the copy pairs, in order;
+ * *num_copies  : how many were written (0 .. num_writes).
+ * Errors: ATTN_EINVAL for a NULL pointer or negative size, a write outside
+ *         the table, an entry with no block (< 0) or outside
+ *         [0, num_blocks), a referenced block with a count below 1, or a
+ *         "free" block out of range or still referenced; ATTN_ENOBLOCKS when
+ *         the free list runs out.  On any error every array is left as it
+ *         was (the batch is all or nothing) and *num_copies is 0.
+ */
+ATTN_API attn_status paged_cow_plan(int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                                    int32_t *ref_counts, int num_blocks, int32_t *free_list, int32_t *free_count,
+                                    const int32_t *write_seqs, const int32_t *write_blocks, int num_writes,
+                                    int32_t *src_out, int32_t *dst_out, int32_t *num_copies);
 
 /*
  * Synchronise `stream`, read the device int32 at err_flag and return

@@ -19,13 +19,13 @@ __all__ = [
     "ATTN_DEVERR_BLOCK_TABLE", "ATTN_DEVERR_SEQ_LEN", "ATTN_DEVERR_TIMEOUT", "ATTN_DEVERR_INDEX",
     "EXPORTED_SYMBOLS", "paged_kv_append", "paged_block_copy", "paged_attn_decode_gqa", "paged_attn_prefill",
     "attn_quantize_fp8", "attn_fwd_fp8", "paged_attn_decode_gqa_workspace_size", "attn_selftest_wait_timeout",
-    "attn_selftest_exp2_poly",
+    "attn_selftest_exp2_poly", "paged_cow_plan",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libattn_sm100.so")
 
-ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_ECUDA, ATTN_EDEVICE = range(5)
+ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_ECUDA, ATTN_EDEVICE, ATTN_ENOBLOCKS = range(6)
 ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_DEVERR_BLOCK_TABLE, ATTN_DEVERR_SEQ_LEN, ATTN_DEVERR_TIMEOUT, ATTN_DEVERR_INDEX = 1, 2, 4, 8
 
@@ -35,7 +35,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "paged_attn_decode_workspace_size", "paged_attn_
                     "paged_attn_decode", "paged_attn_decode_gqa", "paged_attn_decode_noalloc", "paged_attn_prefill",
                     "attn_quantize_fp8", "attn_fwd_fp8",
                     "paged_kv_append",
-                    "paged_block_copy",
+                    "paged_block_copy", "paged_cow_plan",
                     "attn_read_error", "attn_status_str", "attn_selftest_wait_timeout", "attn_selftest_exp2_poly")
 
 # size of the fixed scratch array paged_attn_decode_noalloc uses (attn.h)
@@ -93,6 +93,8 @@ def load():
     lib.paged_kv_append.restype = c_int
     lib.paged_block_copy.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, vp, vp]
     lib.paged_block_copy.restype = c_int
+    lib.paged_cow_plan.argtypes = [vp, c_int, c_int, vp, c_int, vp, vp, vp, vp, c_int, vp, vp, vp]
+    lib.paged_cow_plan.restype = c_int
     lib.attn_read_error.argtypes = [vp, i32p, vp]
     lib.attn_read_error.restype = c_int
     lib.attn_selftest_wait_timeout.argtypes = [vp, vp, vp]
@@ -479,6 +481,52 @@ def paged_block_copy(k_cache, v_cache, src_blocks, dst_blocks, err_flag=None, st
                                      bs, _dtype_code(k_cache.dtype), _ptr(err_flag), _stream(stream, k_cache.device))
     if st != ATTN_OK:
         raise AttnError(st, "paged_block_copy")
+
+
+def paged_cow_plan(block_table, ref_counts, free_list, free_count, write_seqs, write_blocks):
+    """Copy-on-write planning on the host (include/attn.h): for the pending
+    writes (write_seqs[i], write_blocks[i]), in order, every write into a
+    block shared by several sequences takes a free block from the end of
+    ``free_list[:free_count]``, the writer's entry of ``block_table`` is
+    pointed at it and ``ref_counts`` are adjusted -- in place, on the
+    caller's host arrays (numpy int32, or CPU int32 torch tensors, all
+    contiguous).  Returns (src, dst, free_count): the copies to make with
+    paged_block_copy before the writes, as int32 numpy arrays, and the new
+    number of free blocks.  Raises AttnError (ATTN_ENOBLOCKS when the free
+    list runs out, ATTN_EINVAL for an inconsistent table) with every array
+    left as it was."""
+    import numpy as np
+
+    def host(x, name, ndim):
+        if isinstance(x, torch.Tensor):
+            if x.is_cuda:
+                raise ValueError(f"{name} must be a host array (copy-on-write planning runs on the CPU)")
+            x = x.numpy()
+        if not isinstance(x, np.ndarray) or x.dtype != np.int32 or not x.flags.c_contiguous or x.ndim != ndim:
+            raise ValueError(f"{name} must be a contiguous int32 host array with {ndim} dimension(s)")
+        return x
+
+    bt = host(block_table, "block_table", 2)
+    rc = host(ref_counts, "ref_counts", 1)
+    fl = host(free_list, "free_list", 1)
+    ws = host(write_seqs, "write_seqs", 1)
+    wb = host(write_blocks, "write_blocks", 1)
+    if ws.shape != wb.shape:
+        raise ValueError("write_seqs and write_blocks must have one length")
+    if not 0 <= int(free_count) <= fl.shape[0]:
+        raise ValueError("free_count must be within free_list")
+    n = ws.shape[0]
+    src = np.zeros(max(n, 1), dtype=np.int32)
+    dst = np.zeros(max(n, 1), dtype=np.int32)
+    fc = ctypes.c_int32(int(free_count))
+    nc = ctypes.c_int32(0)
+    addr = lambda a: a.ctypes.data if a.size else None  # noqa: E731
+    st = load().paged_cow_plan(addr(bt), bt.shape[0], bt.shape[1], addr(rc), rc.shape[0], addr(fl),
+                               ctypes.byref(fc), addr(ws), addr(wb), n, src.ctypes.data, dst.ctypes.data,
+                               ctypes.byref(nc))
+    if st != ATTN_OK:
+        raise AttnError(st, "paged_cow_plan")
+    return src[:nc.value].copy(), dst[:nc.value].copy(), int(fc.value)
 
 
 def attn_selftest_wait_timeout(err_flag, result=None, stream=None) -> None:

@@ -228,6 +228,7 @@ const char *attn_status_str(attn_status s) {
         case ATTN_EUNSUPPORTED: return "unsupported configuration";
         case ATTN_ECUDA: return "CUDA error";
         case ATTN_EDEVICE: return "device-side error reported in err_flag";
+        case ATTN_ENOBLOCKS: return "no free block left for a copy-on-write copy";
     }
     return "unknown status";
 }

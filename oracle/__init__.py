@@ -15,6 +15,7 @@ from .attention import (  # noqa: F401
     attention_head,
     attention_online_tiled,
     block_copy,
+    cow_plan,
     gather_paged,
     kv_append,
     merge_partials,

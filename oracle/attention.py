@@ -319,6 +319,59 @@ def block_copy(k_cache, v_cache, src_blocks, dst_blocks):
     return k_out, v_out, skipped
 
 
+def cow_plan(block_table, ref_counts, free_list, writes):
+    """Copy-on-write planning for a batch of pending writes.
+
+    [技术详解] §三 "内存共享机制": blocks shared by several sequences carry a
+    reference count; before a sequence writes into a block whose count is
+    above 1, the block is copied to a free block, the writer's table entry
+    is pointed at the copy and the counts are adjusted, so the other
+    sequences keep the old contents ([区别] Q2 and [实现解析] §2.2 give the
+    table from logical to physical blocks this edits).
+
+    block_table [S, max_blocks] (entries < 0: no block), ref_counts
+    [num_blocks], free_list a stack of free block ids (taken from its end),
+    writes a sequence of (seq, logical block) in the order they happen.
+    Each write, in order: the block p = table[s][lb]; if ref[p] == 1 the
+    sequence owns it and writes in place; otherwise the last free block f is
+    taken, ref[p] -= 1, ref[f] = 1, table[s][lb] = f and the pair (p, f) is
+    emitted (the copy runs before the write).  Returns new arrays (table,
+    counts, free list) and the pairs as (src, dst) lists; the inputs are not
+    modified.  Raises ValueError for a write outside the table, an entry
+    without a block or outside [0, num_blocks), a referenced block with a
+    count below 1, a free block that is out of range or still referenced,
+    or a free list that runs out.
+    """
+    table = np.array(block_table, dtype=np.int64, copy=True)
+    refs = np.array(ref_counts, dtype=np.int64, copy=True)
+    free = [int(b) for b in free_list]
+    S, mb = table.shape
+    nb = refs.shape[0]
+    src, dst = [], []
+    for s, lb in writes:
+        s, lb = int(s), int(lb)
+        if not (0 <= s < S and 0 <= lb < mb):
+            raise ValueError(f"write ({s}, {lb}) outside the table")
+        p = int(table[s, lb])
+        if not 0 <= p < nb:
+            raise ValueError(f"write ({s}, {lb}): no block or block {p} out of range")
+        if refs[p] < 1:
+            raise ValueError(f"block {p} is referenced but its count is {refs[p]}")
+        if refs[p] == 1:
+            continue
+        if not free:
+            raise ValueError("the free list ran out")
+        f = free.pop()
+        if not 0 <= f < nb or refs[f] != 0:
+            raise ValueError(f"free block {f} is out of range or still referenced")
+        refs[p] -= 1
+        refs[f] = 1
+        table[s, lb] = f
+        src.append(p)
+        dst.append(f)
+    return table, refs, free, src, dst
+
+
 def paged_prefill(q, k_cache, v_cache, block_table, seq_lens, cu_q, block_size: int, scale: float, seqs=None):
     """Multi-token paged prefill / append oracle.
 

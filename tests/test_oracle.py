@@ -470,6 +470,95 @@ def test_block_copy_and_copy_on_write():
     np.testing.assert_array_equal(np.delete(g1, 2, axis=1), np.delete(kc[4], 2, axis=1))
 
 
+def _refs_of(table, nb):
+    refs = np.zeros(nb, dtype=np.int64)
+    for b in np.asarray(table).ravel():
+        if b >= 0:
+            refs[b] += 1
+    return refs
+
+
+def test_cow_plan_hand_worked():
+    """The copy-on-write step of the pages worked by hand: sequences 0 and 1
+    share physical block 4 (count 2); sequence 1 writing its logical block 0
+    takes free block 7, points its entry there and leaves block 4 to
+    sequence 0 alone (count 1), which then writes in place: no second copy.
+    A repeated write by sequence 1 finds its own block: no copy either."""
+    table = np.array([[4, 1], [4, 3]])
+    refs = np.array([0, 1, 0, 1, 2, 0, 0, 0, 0, 0])
+    t, r, free, src, dst = oracle.cow_plan(table, refs, [9, 7], [(1, 0), (0, 0), (1, 0)])
+    assert src == [4] and dst == [7] and free == [9]
+    np.testing.assert_array_equal(t, [[4, 1], [7, 3]])
+    np.testing.assert_array_equal(r, [0, 1, 0, 1, 1, 0, 0, 1, 0, 0])
+    np.testing.assert_array_equal(table, [[4, 1], [4, 3]])  # inputs untouched
+    # three sharers: the first two writers copy, the last one owns the block
+    table = np.array([[5], [5], [5]])
+    refs = _refs_of(table, 8)
+    t, r, free, src, dst = oracle.cow_plan(table, refs, [1, 2, 3], [(0, 0), (2, 0), (1, 0)])
+    assert src == [5, 5] and dst == [3, 2] and free == [1]
+    np.testing.assert_array_equal(t, [[3], [5], [2]])
+    np.testing.assert_array_equal(r, _refs_of(t, 8))
+
+
+def test_cow_plan_invariants_and_contents():
+    """Random shared-prefix tables: after the plan the counts are again the
+    number of table references, every written entry is exclusive, unwritten
+    entries keep their blocks, no free block is referenced, and copying the
+    pairs (block_copy) leaves every sequence's logical contents as before."""
+    rng = np.random.default_rng(90)
+    for trial in range(30):
+        S, mb, nb = 6, 5, 64
+        pool = list(rng.permutation(nb))
+        prefix = [pool.pop() for _ in range(2)]
+        table = np.full((S, mb), -1)
+        for s in range(S):
+            n = int(rng.integers(1, mb + 1))
+            for lb in range(n):
+                table[s, lb] = prefix[lb] if lb < 2 and s % 3 else pool.pop()
+        refs = _refs_of(table, nb)
+        free = pool[:]
+        live = [(s, lb) for s in range(S) for lb in range(mb) if table[s, lb] >= 0]
+        writes = [live[i] for i in rng.integers(0, len(live), 12)]
+        t, r, fr, src, dst = oracle.cow_plan(table, refs, free, writes)
+        np.testing.assert_array_equal(r, _refs_of(t, nb))
+        for s, lb in writes:
+            assert r[t[s, lb]] == 1
+        written = set(writes)
+        for s, lb in live:
+            if (s, lb) not in written:
+                assert t[s, lb] == table[s, lb]
+        assert not set(fr) & set(t[t >= 0].tolist())
+        assert len(src) == len(set(dst)) == len(free) - len(fr)
+        kc, vc = _pool(seed=100 + trial, nb=nb)
+        k2, v2, skipped = oracle.block_copy(kc, vc, src, dst)
+        assert skipped == []
+        for s, lb in live:
+            np.testing.assert_array_equal(k2[t[s, lb]], kc[table[s, lb]])
+            np.testing.assert_array_equal(v2[t[s, lb]], vc[table[s, lb]])
+
+
+def test_cow_plan_errors_and_planted_mistake():
+    table = np.array([[4, -1], [4, 3]])
+    refs = _refs_of(table, 8)
+    for writes, free in [([(2, 0)], [7]), ([(0, 1)], [7]), ([(0, 0), (1, 0)], []), ([(0, 0)], [3]),
+                         ([(0, 0)], [9])]:
+        with pytest.raises(ValueError):
+            oracle.cow_plan(table, refs, free, writes)
+    bad = refs.copy()
+    bad[3] = 0
+    with pytest.raises(ValueError):
+        oracle.cow_plan(table, bad, [7], [(1, 1)])
+
+    def no_decrement(table, ref_counts, free_list, writes):  # a plausible slip: the source keeps its count
+        t, r, f, src, dst = oracle.cow_plan(table, ref_counts, free_list, writes)
+        for p in src:
+            r[p] += 1
+        return t, r, f, src, dst
+
+    t, r, _, _, _ = no_decrement(np.array([[5], [5]]), np.array([0, 0, 0, 0, 0, 2]), [1], [(0, 0)])
+    assert not (r == _refs_of(t, 6)).all()
+
+
 def test_paged_decode_grouped_query_heads():
     """Grouped-query decode: query head h reads key/value head h // G.  Pinned
     against the multi-head oracle on a cache whose heads are repeated G times
