@@ -329,10 +329,10 @@ class Decode:
                                    base.block_size, base.scale)
         elif name == "decode_shared_prefix_small":
             # 48 sequences (6 groups) of the shared-prefix workload in a
-            # 4000-block pool (2.1 GB of K/V, above L2): the case profiler
+            # 2400-block pool (1.3 GB of K/V, above L2): the case profiler
             # captures run on
             self.p = W.paged_shared_prefix(device=device, seed=seed, **{**W.DECODE_SHARED_PREFIX, "num_seqs": 48,
-                                                                         "pool": 4000})
+                                                                         "pool": 2400})
         elif name == "decode_uniform_small":
             # 16 sequences of the uniform workload in a 4000-block pool (1 GiB
             # of K/V, still above L2): the case profiler captures run on

@@ -327,6 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             uint32_t ukv = 0;         // K/V tiles loaded so far (ring position)
             uint32_t qc[2] = {0, 0};  // Q tiles loaded so far, per query tile
+            // dense L2 policy: a Q tile is read by one unit only (streamed),
+            // while a head's K/V tiles are re-read by every unit of the head
+            // (kept): without the hints the Q and O streams pushed K/V out of
+            // L2 and K/V was read from DRAM about 1.6 times over at 2k
+            const uint64_t pol_stream = l2_policy_evict_first(), pol_keep = l2_policy_evict_last();
             for (int r = 0; ok; ++r) {
                 const int u = snake_unit(r, c, G, n_units);
                 if (u < 0) break;
@@ -348,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_2d(dst + b * kBoxBytes, &tmQ, &q_full[i], x.head * D + b * kBoxCols,
                                             x.qtok0 + x.qrow0 + i * BM);
                             else
-                                tma_load_3d(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols, x.qrow0 + i * BM,
-                                            x.head);
+                                tma_load_3d_hint(dst + b * kBoxBytes, &tmQ, &q_full[i], b * kBoxCols,
+                                                 x.qrow0 + i * BM, x.head, pol_stream);
                         }
                     }
                     __syncwarp();
@@ -379,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (elect_one()) {
                             mbar_arrive_expect_tx(&kv_full[slot], qk ? kQKBytes : C::kTileBytes);
                             for (int b = 0; b < (qk ? kQKBoxes : C::kBoxes); ++b)
-                                tma_load_3d(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols, (v >> 1) * BN,
-                                            x.head);
+                                tma_load_3d_hint(dst + b * kBoxBytes, tm, &kv_full[slot], b * kBoxCols,
+                                                 (v >> 1) * BN, x.head, pol_keep);
                         }
                     } else {
                         // one box per cache block: lane k loads block k of the tile.
@@ -743,8 +748,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     tma_store_2d(&tmO, smem + C::kStageOff + h * kBoxBytes, x.head * D + 64 * h,
                                                  x.qtok0 + tile_row0);
                                 else
-                                    tma_store_3d(&tmO, smem + C::kStageOff + h * kBoxBytes, 64 * h, tile_row0,
-                                                 x.head);
+                                    tma_store_3d_hint(&tmO, smem + C::kStageOff + h * kBoxBytes, 64 * h,
+                                                      tile_row0, x.head, l2_policy_evict_first());
                             }
                             bulk_commit();
                             bulk_wait_read_all();
