@@ -106,6 +106,30 @@ def test_bf16_late_score_jump(causal):
     check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"late score jump causal={causal}")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("keys", ["tile", "poly_column", "sfu_column", "both_halves"])
+def test_bf16_extreme_score_jump(causal, keys):
+    """Keys that score ~141 nats (~204 in log2 units) above the rest: a whole
+    key tile from position 384 on, or single keys at positions 394 and 906
+    (columns 10 of their tiles, exponentiated on the FMA pipe) or 384 (column
+    0, special-function unit), or one in each 128-row half of a query block.
+    Exponentials of those tiles against the running max carried from earlier
+    tiles would overflow fp32, so the running max must move to the new tile's
+    row max before any of them is taken, whichever unit (special-function or
+    FMA pipe) takes it.  The result is still the plain definition's."""
+    inp = W.dense_inputs(1, 2, 1000, 128, dtype=torch.bfloat16, seed=12, device="cuda", causal=causal)
+    Q, K = inp["Q"].clone(), inp["K"].clone()
+    Q[..., 0] = 4.0
+    sel = {"tile": slice(384, 512), "poly_column": [394, 906], "sfu_column": [384],
+           "both_halves": [394, 522]}[keys]
+    K[..., sel, 0] = 400.0
+    inp["Q"], inp["K"] = Q.contiguous(), K.contiguous()
+    O, LSE = _run(inp)
+    O_ref, L_ref = _full_oracle(inp)
+    assert L_ref[..., 600:].min() > 130.0
+    check_close(O, LSE, O_ref, L_ref, torch.bfloat16, f"extreme score jump {keys} causal={causal}")
+
+
 def test_prefill_2k_causal_full_size():
     """B=4 H=16 N=2048 d=128 causal bf16, seed 0: the launch the bench times.
     Four (b, h) heads against the oracle in full; every head for finiteness."""
