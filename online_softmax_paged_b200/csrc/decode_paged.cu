@@ -1102,17 +1102,47 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 // log2-sum-exp and bad flag of partials j, j + 32, ...; the maximum and the
 // weight sum are warp reductions and the weighted rows are summed in partial
 // order, so the result depends only on the lengths and sizes.  The first 16
-// partial rows are requested together with the log2-sum-exps.
+// partial rows are requested together with the log2-sum-exps.  When the
+// tile kernel planned for itself, the row's place in the schedule follows
+// from seq_lens alone (an input, written before that kernel started), so it
+// is worked out before the wait and only the partials are read after it.
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) {
     constexpr int kBatch = 16;  // partial rows in flight per lane
-    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long sh = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (sh >= (long long)a.num_seqs * a.H) return;
-    const int s = (int)(sh / a.H), hq = (int)(sh - (long long)s * a.H);
+    const bool have = sh < (long long)a.num_seqs * a.H;
+    const int s = have ? (int)(sh / a.H) : 0, hq = have ? (int)(sh - (long long)s * a.H) : 0;
+    int st0 = 0, st1 = 0, stn = 0;
+    if (a.fused_plan && have) {
+        // the plan's exclusive prefix at s and s + 1 and its total: tiles of
+        // each sequence (none for an empty or invalid length), summed by the warp
+        int before = 0, upto = 0, all = 0;
+        for (int k = lane; k < a.num_seqs; k += 32) {
+            const int L = __ldg(a.seq_lens + k);
+            const int t = (L > 0 && seq_len_ok(L, a)) ? (L + kTileTok - 1) / kTileTok : 0;
+            all += t;
+            if (k < s) before += t;
+            if (k <= s) upto += t;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            before += __shfl_xor_sync(0xffffffffu, before, o);
+            upto += __shfl_xor_sync(0xffffffffu, upto, o);
+            all += __shfl_xor_sync(0xffffffffu, all, o);
+        }
+        st0 = before;
+        st1 = upto;
+        stn = all;
+    }
+    pdl_wait();
+    if (!have) return;
     const int h = hq / G, g = hq - h * G;
-    const int32_t *starts = a.item_start;
-    const int st0 = __ldcg(starts + s), st1 = __ldcg(starts + s + 1), stn = __ldcg(starts + a.num_seqs);
+    if (!a.fused_plan) {
+        const int32_t *starts = a.item_start;
+        st0 = __ldcg(starts + s);
+        st1 = __ldcg(starts + s + 1);
+        stn = __ldcg(starts + a.num_seqs);
+    }
     const int nts = st1 - st0;
     if (nts == 0) return;  // empty or invalid length: written with the plan
     Sched sc;
