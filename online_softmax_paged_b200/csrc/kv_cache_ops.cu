@@ -10,8 +10,10 @@
 // FlashAttention-2 与 PagedAttention 实现解析" section 2.2 (block table lookup).
 //
 // Both are pure data movement (HBM-bound): 16-byte vector loads and stores,
-// one CTA per token (append); the copy runs grid-stride over 16 KiB chunks of
-// (pair, K|V) so the last wave is a fraction of a chunk, not of a block.
+// each thread issuing all its loads of a round before its first store (4
+// per thread per token for the append, 8 for the copy); one CTA per token
+// (append); the copy runs grid-stride over 32 KiB chunks of (pair, K|V) so
+// the last wave is a fraction of a chunk, not of a block.
 // Out-of-range ids are skipped on the device and reported through err_flag,
 // never dereferenced.
 #include <cuda_runtime.h>
@@ -32,6 +34,8 @@ struct AppendArgs {
     int num_seqs, max_blocks, num_blocks, H, block_size;
     int row_bytes;  // d * element size (a multiple of 16)
 };
+
+constexpr int kAppendUnroll = 4;
 
 __global__ void __launch_bounds__(256) kv_append_kernel(AppendArgs a) {
     __shared__ long long dst_row;  // element row index of (phys, h = 0, slot), or -1
@@ -56,14 +60,29 @@ __global__ void __launch_bounds__(256) kv_append_kernel(AppendArgs a) {
     if (r0 < 0) return;
     const int cpr = a.row_bytes / 16;  // 16-byte chunks per head row
     const int per = a.H * cpr;
-    for (int c = threadIdx.x; c < 2 * per; c += blockDim.x) {
-        const int which = c >= per;
-        const int rem = c - which * per;
-        const int h = rem / cpr, q = rem - h * cpr;
-        const uint8_t *src = (which ? a.v_new : a.k_new) + ((size_t)t * a.H + h) * a.row_bytes + 16 * q;
-        uint8_t *dst = (which ? a.v_cache : a.k_cache) +
-                       ((size_t)r0 + (size_t)h * a.block_size) * a.row_bytes + 16 * q;
-        *reinterpret_cast<uint4 *>(dst) = __ldg(reinterpret_cast<const uint4 *>(src));
+    // kAppendUnroll chunks per thread per round, all loads issued before the
+    // first store (a token is 2 H d-element rows: 16 KiB at H = 32, d = 128,
+    // one round of 256 threads)
+    for (int c0 = threadIdx.x; c0 < 2 * per; c0 += kAppendUnroll * blockDim.x) {
+        uint4 x[kAppendUnroll];
+        uint8_t *dst[kAppendUnroll];
+#pragma unroll
+        for (int u = 0; u < kAppendUnroll; ++u) {
+            const int c = c0 + u * blockDim.x;
+            dst[u] = nullptr;
+            if (c < 2 * per) {
+                const int which = c >= per;
+                const int rem = c - which * per;
+                const int h = rem / cpr, q = rem - h * cpr;
+                const uint8_t *src = (which ? a.v_new : a.k_new) + ((size_t)t * a.H + h) * a.row_bytes + 16 * q;
+                dst[u] = (which ? a.v_cache : a.k_cache) + ((size_t)r0 + (size_t)h * a.block_size) * a.row_bytes +
+                         16 * q;
+                x[u] = __ldg(reinterpret_cast<const uint4 *>(src));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kAppendUnroll; ++u)
+            if (dst[u]) *reinterpret_cast<uint4 *>(dst[u]) = x[u];
     }
 }
 
@@ -73,14 +92,15 @@ struct CopyArgs {
     int32_t *err;
     int num_blocks, num_pairs;
     long long block_bytes;  // H * block_size * d * element size (a multiple of 16)
-    int chunks;             // 16 KiB chunks per block (the last one may be short)
+    int chunks;             // 32 KiB chunks per block (the last one may be short)
 };
 
 constexpr int kCopyThreads = 256;
-constexpr int kChunkBytes = kCopyThreads * 4 * 16;  // 4 x 16 bytes in flight per thread
+constexpr int kCopyUnroll = 8;                                 // 16-byte words in flight per thread
+constexpr int kChunkBytes = kCopyThreads * kCopyUnroll * 16;  // 32 KiB
 
 // Work unit w: pair w / (2 chunks), K (0) or V (1), chunk; each thread moves
-// 4 x 16 bytes with all four loads issued before the first store.
+// kCopyUnroll x 16 bytes with all loads issued before the first store.
 __global__ void __launch_bounds__(kCopyThreads) block_copy_kernel(CopyArgs a) {
     const long long units = (long long)a.num_pairs * 2 * a.chunks;
     for (long long w = blockIdx.x; w < units; w += gridDim.x) {
@@ -99,12 +119,11 @@ __global__ void __launch_bounds__(kCopyThreads) block_copy_kernel(CopyArgs a) {
         uint4 *to = reinterpret_cast<uint4 *>(base + (size_t)d * a.block_bytes + off);
         const int t = threadIdx.x;
         if (n == kChunkBytes / 16) {
-            const uint4 x0 = from[t], x1 = from[t + kCopyThreads], x2 = from[t + 2 * kCopyThreads],
-                        x3 = from[t + 3 * kCopyThreads];
-            to[t] = x0;
-            to[t + kCopyThreads] = x1;
-            to[t + 2 * kCopyThreads] = x2;
-            to[t + 3 * kCopyThreads] = x3;
+            uint4 x[kCopyUnroll];
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) x[u] = from[t + u * kCopyThreads];
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) to[t + u * kCopyThreads] = x[u];
         } else {
             for (long long k = t; k < n; k += kCopyThreads) to[k] = from[k];
         }
