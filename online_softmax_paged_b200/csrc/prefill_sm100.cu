@@ -158,12 +158,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
 
 
 // Pairs k with (k % 8) >= kPolyFrom take the polynomial; the others MUFU ex2.
-constexpr int kPolyFrom = 5;  // 3 of every 8 pairs
+constexpr int kPolyFrom = 6;  // 2 of every 8 pairs (re-measured against 1 and 3 of 8)
 
 // P = 2^(s * scale_log2 - m) for one 128-wide score row held as raw fp32 bits
 // in sr, packed to bf16 pairs and stored over the first 64 TMEM columns of
 // the row's S region; the fp32 values are summed into acc2 (4 pairs of
-// accumulators).  USE_POLY sends 3 of every 8 pairs to the FMA-pipe
+// accumulators).  USE_POLY sends 2 of every 8 pairs to the FMA-pipe
 // polynomial (only for tiles without masked entries).
 template <bool USE_POLY>
 __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint32_t s_tm, uint64_t scale2,
