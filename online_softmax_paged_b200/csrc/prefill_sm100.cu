@@ -163,9 +163,11 @@ constexpr int kPolyFrom = 6;  // 2 of every 8 pairs (re-measured against 1 and 3
 // P = 2^(s * scale_log2 - m) for one 128-wide score row held as raw fp32 bits
 // in sr, packed to bf16 pairs and stored over the first 64 TMEM columns of
 // the row's S region; the fp32 values are summed into acc2 (4 pairs of
-// accumulators).  USE_POLY sends 2 of every 8 pairs to the FMA-pipe
-// polynomial (only for tiles without masked entries).
-template <bool USE_POLY>
+// accumulators).  2 of every 8 pairs go to the FMA-pipe polynomial, masked
+// tiles included: a masked score (-inf) comes out of its clamp as 2^-125
+// instead of 0, which adds nothing visible to a running sum l >= 1 or to O
+// (the V rows under masked keys are finite: real keys, zero-filled rows
+// past N, and the zeroed dead rows of a paged sequence's last tile).
 __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint32_t s_tm, uint64_t scale2,
                                                uint64_t negm2, uint64_t (&acc2)[4]) {
     // one 32-score chunk at a time: its 16 packed words are stored before the
@@ -178,7 +180,7 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], uint
             const uint64_t x2 =
                 f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), scale2, negm2);
             uint64_t p2;
-            if (USE_POLY && ((e + 16 * c) & 7) >= kPolyFrom) {
+            if (((e + 16 * c) & 7) >= kPolyFrom) {
                 p2 = exp2_poly2(x2);
             } else {
                 float x0, x1;
@@ -678,10 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t scale2 = f2_pack(c_step, c_step);
                 const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
                 uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-                if (masked)
-                    exp_pack_store<false>(sr, s_tm, scale2, negm2, acc2);
-                else
-                    exp_pack_store<true>(sr, s_tm, scale2, negm2, acc2);
+                exp_pack_store(sr, s_tm, scale2, negm2, acc2);
                 float psum;
                 {
                     const uint64_t t2 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
