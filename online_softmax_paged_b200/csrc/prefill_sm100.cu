@@ -157,6 +157,24 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
 // ---------------------------------------------------------------- softmax math
 
 
+// 32 lanes x 64 consecutive 32-bit columns in one load: columns 0-31 of the
+// group to lo, 32-63 to hi (thread t gets lane base + t).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&lo)[32], uint32_t (&hi)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : "=r"(lo[0]), "=r"(lo[1]), "=r"(lo[2]), "=r"(lo[3]), "=r"(lo[4]), "=r"(lo[5]), "=r"(lo[6]), "=r"(lo[7]),
+          "=r"(lo[8]), "=r"(lo[9]), "=r"(lo[10]), "=r"(lo[11]), "=r"(lo[12]), "=r"(lo[13]), "=r"(lo[14]), "=r"(lo[15]),
+          "=r"(lo[16]), "=r"(lo[17]), "=r"(lo[18]), "=r"(lo[19]), "=r"(lo[20]), "=r"(lo[21]), "=r"(lo[22]), "=r"(lo[23]),
+          "=r"(lo[24]), "=r"(lo[25]), "=r"(lo[26]), "=r"(lo[27]), "=r"(lo[28]), "=r"(lo[29]), "=r"(lo[30]), "=r"(lo[31]),
+          "=r"(hi[0]), "=r"(hi[1]), "=r"(hi[2]), "=r"(hi[3]), "=r"(hi[4]), "=r"(hi[5]), "=r"(hi[6]), "=r"(hi[7]),
+          "=r"(hi[8]), "=r"(hi[9]), "=r"(hi[10]), "=r"(hi[11]), "=r"(hi[12]), "=r"(hi[13]), "=r"(hi[14]), "=r"(hi[15]),
+          "=r"(hi[16]), "=r"(hi[17]), "=r"(hi[18]), "=r"(hi[19]), "=r"(hi[20]), "=r"(hi[21]), "=r"(hi[22]), "=r"(hi[23]),
+          "=r"(hi[24]), "=r"(hi[25]), "=r"(hi[26]), "=r"(hi[27]), "=r"(hi[28]), "=r"(hi[29]), "=r"(hi[30]), "=r"(hi[31])
+        : "r"(taddr));
+}
+
 // Pairs k with (k % 8) >= kPolyFrom take the polynomial; the others MUFU ex2.
 constexpr int kPolyFrom = 6;  // 2 of every 8 pairs (re-measured against 1 and 3 of 8)
 
@@ -639,8 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t sr[4][32];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_tm + 32 * cc, sr[cc]);
+                tmem_ld64(s_tm, sr[0], sr[1]);  // the score row in two 64-column loads
+                tmem_ld64(s_tm + 64, sr[2], sr[3]);
                 tmem_wait_ld();
                 // visible keys: col <= lim; only key tiles reaching past the
                 // tile's first row position (the causal diagonal) and the
