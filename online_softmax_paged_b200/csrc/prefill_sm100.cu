@@ -273,8 +273,8 @@ __device__ __forceinline__ void get_unit(const PrefillArgs &a, bool causal, int 
     // the extra (diagonal) step is the one it serves first: once that step's
     // P.V is issued the next unit's first QK^T products follow at once,
     // instead of tile 0 waiting behind tile 1's extra softmax (+2.5-3 % at
-    // 2k, measured; the FP8 mode, whose QK^T is twice as fast, measured
-    // 1.5 % slower with it and keeps the plain order).
+    // 2k, measured; the FP8 mode, whose QK^T is twice as fast, measured it
+    // neutral and keeps the plain order).
     x.row0[0] = x.qrow0 + (later_first ? BM : 0);
     x.row0[1] = x.qrow0 + (later_first ? 0 : BM);
     int n[NQ];
