@@ -24,8 +24,10 @@
 //     key tile: PV0(j), S0(j+1), PV1(j), S1(j+1): while one softmax
 //     warpgroup exponentiates, the tensor core works on the other tile.
 //   * Warps 0-3 / 4-7 (softmax, one thread per query row): tcgen05.ld the
-//     score row, causal / length mask, row max, exp2, bf16 P written back over
-//     the scores in TMEM, running sum.  The reference max only moves when the
+//     score row (two 64-column loads), causal / length mask, row max, exp2
+//     (2 of every 8 pairs by an FMA-pipe polynomial, the rest on the
+//     special-function unit), bf16 P written back over the scores in TMEM,
+//     running sum.  The reference max only moves when the
 //     row max grows by more than 2^8 (exact: P and l use the same stale max;
 //     the O accumulator is rescaled only then).  Epilogue: O / l, bf16 store,
 //     LSE = (m + log2 l) ln 2.
