@@ -1104,8 +1104,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 // order, so the result depends only on the lengths and sizes.  The first 16
 // partial rows are requested together with the log2-sum-exps.  When the
 // tile kernel planned for itself, the row's place in the schedule follows
-// from seq_lens alone (an input, written before that kernel started), so it
-// is worked out before the wait and only the partials are read after it.
+// from seq_lens alone, so it is worked out before the wait and only the
+// partials are read after it.  seq_lens is an input: this grid starts only
+// once every CTA of the tile kernel has passed that kernel's own dependency
+// wait, so whatever wrote seq_lens before the call has completed.
 __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeArgs a, int G) {
     constexpr int kBatch = 16;  // partial rows in flight per lane
     const int lane = threadIdx.x & 31;
