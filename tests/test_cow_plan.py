@@ -156,3 +156,72 @@ def test_copy_on_write_append_then_decode():
     # the sharers that did not copy still read the old prefix blocks
     O_ref, L_ref = oracle.paged_decode(q.double().numpy(), k3, v3, t_ref, lens + 1, bs, 1.0 / np.sqrt(d))
     check_close(O, LSE, O_ref, L_ref, torch.bfloat16, "copy-on-write append + decode")
+
+
+def _random_state(data_seed):
+    """A random, mostly consistent block pool: shared and private blocks in a
+    table, the counts of its references, the unused blocks as a shuffled free
+    list (sometimes cut short), and a batch of writes that are mostly to
+    entries holding a block, sometimes outside the table or to empty entries."""
+    rng = np.random.default_rng(data_seed)
+    S, mb, nb = int(rng.integers(1, 7)), int(rng.integers(1, 6)), int(rng.integers(4, 41))
+    table = np.full((S, mb), -1, dtype=np.int32)
+    pool = [int(b) for b in rng.permutation(nb)]
+    shared = [pool.pop() for _ in range(int(rng.integers(0, min(4, len(pool)) + 1)))]
+    for s in range(S):
+        for lb in range(int(rng.integers(0, mb + 1))):
+            if shared and rng.random() < 0.5:
+                table[s, lb] = shared[int(rng.integers(0, len(shared)))]
+            elif pool:
+                table[s, lb] = pool.pop()
+    refs = np.zeros(nb, dtype=np.int32)
+    for b in table[table >= 0]:
+        refs[b] += 1
+    free = np.array(pool[:int(rng.integers(0, len(pool) + 1))], dtype=np.int32)
+    live = [(s, lb) for s in range(S) for lb in range(mb) if table[s, lb] >= 0]
+    writes = []
+    for _ in range(int(rng.integers(0, 12))):
+        u = rng.random()
+        if live and u < 0.9:
+            writes.append(live[int(rng.integers(0, len(live)))])
+        else:
+            writes.append((int(rng.integers(-1, S + 1)), int(rng.integers(-1, mb + 1))))
+    return table, refs, free, writes
+
+
+@pytest.mark.parametrize("seed", range(200))
+def test_planner_random_batches_match_oracle(seed):
+    """Random pools and batches, some of them invalid or short of free
+    blocks: the library succeeds exactly when the oracle does, with the same
+    table, counts, free list and copy pairs; when it fails it leaves every
+    array as it was (all or nothing), and a batch whose writes are all valid
+    but which runs out of free blocks reports ATTN_ENOBLOCKS."""
+    osp = _osp()
+    table, refs, free, writes = _random_state(1000 + seed)
+    try:
+        expect = oracle.cow_plan(table, refs, list(free), writes)
+        err = None
+    except ValueError as e:
+        expect, err = None, str(e)
+    t, r, f = table.copy(), refs.copy(), free.copy()
+    ws = np.array([w[0] for w in writes], dtype=np.int32)
+    wb = np.array([w[1] for w in writes], dtype=np.int32)
+    if expect is not None:
+        src, dst, fc = osp.paged_cow_plan(t, r, f, len(f), ws, wb)
+        t_ref, r_ref, f_ref, src_ref, dst_ref = expect
+        assert src.tolist() == src_ref and dst.tolist() == dst_ref
+        np.testing.assert_array_equal(t, t_ref)
+        np.testing.assert_array_equal(r, r_ref)
+        assert f[:fc].tolist() == f_ref
+    else:
+        with pytest.raises(osp.AttnError) as e:
+            osp.paged_cow_plan(t, r, f, len(f), ws, wb)
+        np.testing.assert_array_equal(t, table)
+        np.testing.assert_array_equal(r, refs)
+        np.testing.assert_array_equal(f, free)
+        S, mb = table.shape
+        all_valid = all(0 <= s < S and 0 <= lb < mb and table[s, lb] >= 0 for s, lb in writes)
+        if all_valid and "ran out" in err:
+            assert e.value.status == osp.ATTN_ENOBLOCKS
+        else:
+            assert e.value.status in (1, osp.ATTN_ENOBLOCKS)
